@@ -1,0 +1,278 @@
+"""fp64 CPU oracle for absorbed multi-head latent attention (MLA).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke entry and the CPU-baseline leg of the
+benchmark may import this module.  The library's GPU path never calls it and shares no code
+with it; this file imports nothing but numpy.
+
+Every function follows one passage of the source pages and is written as the plain definition,
+in float64, with no intermediate rounding (the pages round to bf16 after each Linear/einsum; the
+GPU path rounds at similar points and the parity tolerance absorbs it).  Library primitives used
+as steps: numpy ``matmul``/``einsum`` (contractions), ``exp``/``log``/``sqrt``/``sin``/``cos``.
+
+Source pages (cited by title and section):
+  [QRMS]  DeepSeek V4.1 · Query RMSNorm — formula block and the ``RMSNorm`` excerpt.
+  [QH]    DeepSeek-V3.2-Exp · Query heads — the six-step formula block, the parameter table, the
+          "Explanation" (one wq_b, split per head after the product), the ``mla-init`` and
+          ``mla-queries`` excerpts.
+  [AU]    DeepSeek-V3.2-Exp · Attention update — ``block``, ``rmsnorm`` (residual form) and the
+          ``mla-decode`` (absorbed "MQA decode") excerpts.
+  [VS]    Kimi-K2 · value_states — parameter table, ``mla-init`` and ``mla-prefill`` excerpts
+          (the non-absorbed form: rebuilt per-head keys/values, additive causal mask).
+
+Readings where the pages are silent or garbled (each also listed in the design notes):
+  * RoPE is the interleaved kind (adjacent pairs (2i, 2i+1)); base theta = 10000;
+    theta_i = theta^(-2i/rope_dim); positive rotation (x0 cos - x1 sin, x0 sin + x1 cos).
+  * The pe cache holds keys that are already rotated (the cache producer is off the path).
+  * The index mask of the V3.2 decode excerpt is taken with top-k >= end_pos, i.e. dense.
+  * Decode query sits at position start_pos and sees keys 0..start_pos; a prefill query t sees
+    keys 0..start_pos+t.
+  * softmax_scale = qk_head_dim^-0.5 (the YaRN mscale branch of [QH] mla-init is off).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "rmsnorm", "rope_frequencies", "apply_rope_interleaved", "query_heads", "absorb_w_uk",
+    "latent_scores", "softmax_fp", "latent_weighted_sum", "expand_w_uv", "decode", "prefill",
+    "nonabsorbed_attention", "split_wkv_b", "split_wq_b",
+]
+
+
+# ------------------------------------------------------------------------------------------
+# a1: RMSNorm with optional residual  ([AU] rmsnorm; [QRMS] formula and excerpt)
+# ------------------------------------------------------------------------------------------
+def rmsnorm(x: np.ndarray, gamma: np.ndarray, eps: float = 1e-6,
+            residual: np.ndarray | None = None):
+    """y = gamma * u / sqrt(mean_j(u_j^2) + eps) over the last axis, u = x (+ residual).
+
+    With a residual, the pages first add it (``x = residual = x + residual``) and return the
+    sum as the new residual.  Returns ``(y, u_or_None)``.
+    """
+    u = np.asarray(x, dtype=np.float64)
+    if residual is not None:
+        u = u + np.asarray(residual, dtype=np.float64)
+    m2 = np.mean(u * u, axis=-1, keepdims=True)
+    y = np.asarray(gamma, dtype=np.float64) * (u / np.sqrt(m2 + eps))
+    return y, (u if residual is not None else None)
+
+
+# ------------------------------------------------------------------------------------------
+# a3: interleaved rotary embedding  ([QH] step "Q^R_t = RoPE(Q^pe_t, R_t)", R [T, 32 pairs])
+# ------------------------------------------------------------------------------------------
+def rope_frequencies(rope_dim: int, theta: float = 10000.0) -> np.ndarray:
+    """theta_i = theta^(-2i/rope_dim), i < rope_dim/2 (one angle rate per pair)."""
+    i = np.arange(rope_dim // 2, dtype=np.float64)
+    return np.power(float(theta), -2.0 * i / rope_dim)
+
+
+def apply_rope_interleaved(x: np.ndarray, pos: np.ndarray, theta: float = 10000.0) -> np.ndarray:
+    """Rotate each adjacent pair (x[2i], x[2i+1]) of the last axis by angle pos * theta_i.
+
+    ``x`` is [..., rope_dim]; ``pos`` broadcasts against ``x.shape[:-1]``.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    rope_dim = x.shape[-1]
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * rope_frequencies(rope_dim, theta)
+    c, s = np.cos(ang), np.sin(ang)
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    out = np.empty(np.broadcast_shapes(x.shape, ang.shape[:-1] + (rope_dim,)), dtype=np.float64)
+    out[..., 0::2] = x0 * c - x1 * s
+    out[..., 1::2] = x0 * s + x1 * c
+    return out
+
+
+# ------------------------------------------------------------------------------------------
+# a2-a3: query heads  ([QH] formula block, Explanation, mla-queries excerpt)
+# ------------------------------------------------------------------------------------------
+def split_wq_b(wq_b: np.ndarray, n_heads: int, nope: int, rope: int):
+    """View wq_b [H*(nope+rope), q_lora] per head and return (W_UQ rows, W_QR rows):
+    [H, nope, q_lora] and [H, rope, q_lora].  Each head's block is nope content rows followed by
+    rope rows ([QH] Explanation: one matrix, split per head after the product)."""
+    w = np.asarray(wq_b, dtype=np.float64).reshape(n_heads, nope + rope, -1)
+    return w[:, :nope, :], w[:, nope:, :]
+
+
+def query_heads(y: np.ndarray, wq_b: np.ndarray, n_heads: int, nope: int, rope: int,
+                pos: np.ndarray, theta: float = 10000.0):
+    """q = y @ wq_b^T viewed [M, H, nope+rope]; q_nope = first nope features of each head,
+    q_pe = RoPE(last rope features).  ``y`` is [M, q_lora]; ``pos`` is [M]."""
+    q = np.asarray(y, dtype=np.float64) @ np.asarray(wq_b, dtype=np.float64).T
+    q = q.reshape(q.shape[0], n_heads, nope + rope)
+    q_nope = q[..., :nope]
+    q_pe = apply_rope_interleaved(q[..., nope:], np.asarray(pos)[:, None], theta)
+    return q_nope, q_pe
+
+
+# ------------------------------------------------------------------------------------------
+# a4-a8: absorbed attention  ([AU] mla-decode excerpt)
+# ------------------------------------------------------------------------------------------
+def split_wkv_b(wkv_b: np.ndarray, n_heads: int, nope: int, v: int):
+    """wkv_b [H*(nope+v), kv_lora] viewed [H, nope+v, kv_lora]: W_UK = the first nope rows of each
+    head, W_UV = the last v rows ([AU] mla-decode: ``wkv_b[:, :nope]`` and ``wkv_b[:, -v:]``)."""
+    w = np.asarray(wkv_b, dtype=np.float64).reshape(n_heads, nope + v, -1)
+    return w[:, :nope, :], w[:, nope:, :]
+
+
+def absorb_w_uk(q_nope: np.ndarray, w_uk: np.ndarray) -> np.ndarray:
+    """q_lat[m, h, c] = sum_d q_nope[m, h, d] * W_UK[h, d, c]  ("bshd,hdc->bshc")."""
+    return np.einsum("mhd,hdc->mhc", np.asarray(q_nope, np.float64), w_uk)
+
+
+def latent_scores(q_lat: np.ndarray, q_pe: np.ndarray, kv: np.ndarray, pe: np.ndarray,
+                  scale: float) -> np.ndarray:
+    """s[h, t] = (q_lat[h]·kv[t] + q_pe[h]·pe[t]) * scale for one query row.
+
+    ``q_lat`` [H, kv_lora], ``q_pe`` [H, rope], ``kv`` [keys, kv_lora], ``pe`` [keys, rope]."""
+    return (q_lat @ kv.T + q_pe @ pe.T) * scale
+
+
+def softmax_fp(s: np.ndarray):
+    """Softmax along the last axis with max subtraction; also returns lse = log sum exp(s)."""
+    m = np.max(s, axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    z = np.sum(e, axis=-1, keepdims=True)
+    return e / z, (m + np.log(z))[..., 0]
+
+
+def latent_weighted_sum(p: np.ndarray, kv: np.ndarray) -> np.ndarray:
+    """o_lat[h, c] = sum_t p[h, t] * kv[t, c]  ("bsht,btc->bshc")."""
+    return p @ kv
+
+
+def expand_w_uv(o_lat: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
+    """out[..., h, d] = sum_c o_lat[..., h, c] * W_UV[h, d, c]  ("bshc,hdc->bshd")."""
+    return np.einsum("...hc,hdc->...hd", o_lat, w_uv)
+
+
+def _attend_row(q_lat_h, q_pe_h, kv, pe, scale, w_uv, want_logits=False):
+    s = latent_scores(q_lat_h, q_pe_h, kv, pe, scale)
+    p, lse = softmax_fp(s)
+    o_lat = latent_weighted_sum(p, kv)
+    out = expand_w_uv(o_lat, w_uv)
+    return out, lse, (s if want_logits else None), o_lat
+
+
+def _front(q_latent_rows, residual_rows, gamma, wq_b, wkv_b, dims, pos, theta, eps):
+    H, nope, rope, v = dims["n_heads"], dims["nope"], dims["rope"], dims["v"]
+    y, res = rmsnorm(q_latent_rows, gamma, eps, residual_rows)
+    q_nope, q_pe = query_heads(y, wq_b, H, nope, rope, pos, theta)
+    w_uk, w_uv = split_wkv_b(wkv_b, H, nope, v)
+    q_lat = absorb_w_uk(q_nope, w_uk)
+    return y, res, q_nope, q_pe, q_lat, w_uv
+
+
+def _dims(n_heads, nope=128, rope=64, v=128):
+    return {"n_heads": n_heads, "nope": nope, "rope": rope, "v": v}
+
+
+def decode(q_latent, gamma, wq_b, wkv_b, cache, start_pos, n_heads, *, residual=None,
+           kv_lora=512, nope=128, rope=64, v=128, theta=10000.0, eps=1e-6, scale=None,
+           rows=None, want_logits=False, want_intermediates=False):
+    """Absorbed decode ([AU] mla-decode with the index mask keeping every key).
+
+    ``q_latent`` [B, q_lora]; ``cache`` [B, max_t, kv_lora+rope] (packed latents ‖ pe key);
+    ``start_pos`` [B]: sequence b's query is at position start_pos[b] and sees keys 0..start_pos[b].
+    ``rows`` optionally restricts the computation to some sequences.  Returns a dict with
+    ``out`` [R, H, v], ``lse`` [R, H] and, on request, ``logits`` (list of [H, keys]) and the
+    intermediates y, residual_out, q_nope, q_pe, q_lat, o_lat."""
+    rows = np.arange(len(start_pos)) if rows is None else np.asarray(rows)
+    if scale is None:
+        scale = float(nope + rope) ** -0.5
+    dims = _dims(n_heads, nope, rope, v)
+    q_latent = np.asarray(q_latent, np.float64)[rows]
+    res_in = None if residual is None else np.asarray(residual, np.float64)[rows]
+    pos = np.asarray(start_pos)[rows].astype(np.int64)
+    y, res, q_nope, q_pe, q_lat, w_uv = _front(q_latent, res_in, gamma, wq_b, wkv_b, dims,
+                                                pos, theta, eps)
+    outs, lses, logits, olats = [], [], [], []
+    for i, b in enumerate(rows):
+        n = int(pos[i]) + 1
+        kv = np.asarray(cache[b, :n, :kv_lora], np.float64)
+        pe = np.asarray(cache[b, :n, kv_lora:kv_lora + rope], np.float64)
+        o, lse, s, o_lat = _attend_row(q_lat[i], q_pe[i], kv, pe, scale, w_uv, want_logits)
+        outs.append(o)
+        lses.append(lse)
+        logits.append(s)
+        olats.append(o_lat)
+    r = {"out": np.stack(outs), "lse": np.stack(lses)}
+    if want_logits:
+        r["logits"] = logits
+    if want_intermediates:
+        r.update(y=y, residual_out=res, q_nope=q_nope, q_pe=q_pe, q_lat=q_lat,
+                 o_lat=np.stack(olats))
+    return r
+
+
+def prefill(q_latent, gamma, wq_b, wkv_b, cache, start_pos, n_heads, *, residual=None,
+            kv_lora=512, nope=128, rope=64, v=128, theta=10000.0, eps=1e-6, scale=None,
+            batch_rows=None, tokens=None, want_intermediates=False):
+    """Absorbed attention for a chunk of T new tokens after ``start_pos`` (int) cached positions.
+
+    Query t of sequence b is at position start_pos + t and sees keys 0..start_pos+t (causal;
+    the additive mask of [VS] mla-prefill, -inf above the diagonal).  ``q_latent`` [B, T, q_lora];
+    cache rows start_pos..start_pos+T-1 already hold the chunk's own latents.  ``tokens``
+    optionally restricts the computation to some token indices.  Returns ``out`` [B', T', H, v]
+    and ``lse`` [B', T', H]."""
+    q_latent = np.asarray(q_latent, np.float64)
+    B, T, _ = q_latent.shape
+    batch_rows = np.arange(B) if batch_rows is None else np.asarray(batch_rows)
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    if scale is None:
+        scale = float(nope + rope) ** -0.5
+    dims = _dims(n_heads, nope, rope, v)
+    out = np.empty((len(batch_rows), len(tokens), n_heads, v))
+    lse = np.empty((len(batch_rows), len(tokens), n_heads))
+    inter = []
+    for bi, b in enumerate(batch_rows):
+        xs = q_latent[b, tokens]
+        rs = None if residual is None else np.asarray(residual, np.float64)[b, tokens]
+        pos = int(start_pos) + tokens.astype(np.int64)
+        y, res, q_nope, q_pe, q_lat, w_uv = _front(xs, rs, gamma, wq_b, wkv_b, dims, pos,
+                                                    theta, eps)
+        for ti in range(len(tokens)):
+            n = int(pos[ti]) + 1
+            kv = np.asarray(cache[b, :n, :kv_lora], np.float64)
+            pe = np.asarray(cache[b, :n, kv_lora:kv_lora + rope], np.float64)
+            o, l, _, _ = _attend_row(q_lat[ti], q_pe[ti], kv, pe, scale, w_uv)
+            out[bi, ti] = o
+            lse[bi, ti] = l
+        inter.append(dict(y=y, residual_out=res, q_nope=q_nope, q_pe=q_pe, q_lat=q_lat))
+    r = {"out": out, "lse": lse}
+    if want_intermediates:
+        r["intermediates"] = inter
+    return r
+
+
+# ------------------------------------------------------------------------------------------
+# Non-absorbed form  ([VS] mla-prefill: rebuilt per-head keys and values, additive mask)
+# ------------------------------------------------------------------------------------------
+def nonabsorbed_attention(q_nope, q_pe, kv, pe, wkv_b, n_heads, *, q_positions, nope=128,
+                          v=128, scale=None):
+    """Multi-head attention with keys and values rebuilt from the latent cache.
+
+    ``q_nope`` [Tq, H, nope], ``q_pe`` [Tq, H, rope] (rotated); ``kv`` [keys, kv_lora];
+    ``pe`` [keys, rope] is the shared rotary key of every head.  Per head h:
+    k_nope[t] = W_UK[h] kv[t], key[t] = [k_nope[t] ‖ pe[t]], value[t] = W_UV[h] kv[t];
+    weights = softmax(query·key^T·scale + mask) with mask[i, t] = 0 if t <= q_positions[i] else
+    -inf; output = weights · value.  Returns ([Tq, H, v], lse [Tq, H])."""
+    rope = q_pe.shape[-1]
+    if scale is None:
+        scale = float(nope + rope) ** -0.5
+    w_uk, w_uv = split_wkv_b(wkv_b, n_heads, nope, v)
+    kv = np.asarray(kv, np.float64)
+    pe = np.asarray(pe, np.float64)
+    keys_n = kv.shape[0]
+    mask = np.where(np.arange(keys_n)[None, :] <= np.asarray(q_positions)[:, None], 0.0, -np.inf)
+    out = np.empty((q_nope.shape[0], n_heads, v))
+    lse = np.empty((q_nope.shape[0], n_heads))
+    for h in range(n_heads):
+        k_nope = kv @ w_uk[h].T                                   # [keys, nope]
+        key = np.concatenate([k_nope, pe], axis=1)                # [keys, nope+rope]
+        value = kv @ w_uv[h].T                                    # [keys, v]
+        query = np.concatenate([q_nope[:, h], q_pe[:, h]], axis=1)  # [Tq, nope+rope]
+        logits = query @ key.T * scale + mask
+        p, l = softmax_fp(logits)
+        out[:, h] = p @ value
+        lse[:, h] = l
+    return out, lse
