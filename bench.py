@@ -1,0 +1,403 @@
+"""Benchmark of the absorbed-MLA hot path on B200.
+
+One step = one full decode call (q_norm → wq_b+RoPE → W_UK absorption → latent attention over
+the cache → combine → W_UV) for the DeepSeek-V3.2-shaped decode batch: B=32 sequences, H=128,
+cache L=4096 (keys 0..4096), bf16, synthetic seeded inputs resident in HBM.  Between timed steps
+L2 is flushed by writing a 256 MiB buffer (the step's own inputs are 261 MB as well).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+        [--workload v32_decode|kimi_decode|ragged_decode|tiny_decode|prefill_chunk]
+For N > 1 launch one process per GPU with torch.distributed.run; every rank runs its own replica
+batch (the path shards by sequence with no exchange: weak scaling) and rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from mla_synth import keys_per_row, make_inputs, workload  # noqa: E402
+
+METRIC = "MLA decode queries/s + HBM GB/s (% peak); prefill-chunk TFLOP/s (% peak)"
+FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------------------------------
+# Algorithmic work of one step (bytes the method must move, flops it must do)
+# ------------------------------------------------------------------------------------------
+def algorithmic_work(w, start_pos: np.ndarray) -> dict:
+    d = w.dims
+    H, R, C, Dn, Dr, Dv = d.n_heads, d.q_lora_rank, d.kv_lora_rank, d.qk_nope_head_dim, d.qk_rope_head_dim, d.v_head_dim
+    rows = w.batch * w.tokens
+    keys = keys_per_row(w, start_pos)                      # [B, T] visible keys per query row
+    if w.mode == "decode":
+        cache_rows = int(keys.sum())                       # each decode row reads its own keys
+    else:
+        cache_rows = int(keys[:, -1].sum())                # a chunk reads its cache prefix once
+    act = rows * R * 2 * (3 if w.residual else 1) + rows * R * 2   # x (+res r/w) + y
+    weights = H * (Dn + Dr) * R * 2 + H * (Dn + Dv) * C * 2 + R * 4
+    cache = cache_rows * (C + Dr) * 2
+    out = rows * H * Dv * 2
+    flops = (2 * rows * R * H * (Dn + Dr) + 2 * rows * H * Dn * C
+             + 2 * int(keys.sum()) * H * ((C + Dr) + C) + 2 * rows * H * C * Dv)
+    attn_bytes = cache + rows * H * (C + Dr) * 2 + rows * H * C * 2
+    attn_flops = 2 * int(keys.sum()) * H * ((C + Dr) + C)
+    return dict(bytes=act + weights + cache + out, flops=flops, cache_bytes=cache,
+                weight_bytes=weights, attn_bytes=attn_bytes, attn_flops=attn_flops,
+                keys=int(keys.sum()), rows=rows)
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------
+# Our arm
+# ------------------------------------------------------------------------------------------
+def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    dev = f"cuda:{local_rank}"
+    from head_latent_attention_11_b200 import (build, mla_enable_stage_timing,
+                                               mla_last_launch_count, mla_stage_times)
+    build.build()
+    from head_latent_attention_11_b200.runtime import MLARuntime
+
+    w = workload(args.workload)
+    inp = make_inputs(w, seed=args.seed + rank)
+    work = algorithmic_work(w, inp["start_pos"])
+    B, T, H = w.batch, w.tokens, w.dims.n_heads
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q_latent = bf16(inp["q_latent"])
+    if w.mode == "decode":
+        q_latent = q_latent.reshape(B, -1)
+    residual = bf16(inp["residual"]) if inp["residual"] is not None else None
+    if residual is not None and w.mode == "decode":
+        residual = residual.reshape(B, -1)
+    gamma = torch.from_numpy(inp["gamma"]).to(dev)
+    wq_b, wkv_b, cache = bf16(inp["wq_b"]), bf16(inp["wkv_b"]), bf16(inp["cache"])
+    start_pos = torch.from_numpy(inp["start_pos"].astype(np.int32)).to(dev)
+    del inp
+    rt = MLARuntime(gamma, wq_b, wkv_b, n_heads=H, max_rows=B * T, max_seq_len=cache.shape[1],
+                    rope_theta=w.rope_theta, rms_eps=w.rms_eps)
+    out_shape = (B, H, 128) if w.mode == "decode" else (B, T, H, 128)
+    out = torch.empty(out_shape, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        if w.mode == "decode":
+            rt.decode(q_latent, start_pos, cache, residual=residual, out=out)
+        else:
+            rt.prefill(q_latent, w.prefill_start, cache, residual=residual, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if rt.sync_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    # ---- timed region: K steps, L2 flushed before each (flush not timed)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank if world > 1 else int(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or 0))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    launches = mla_last_launch_count(rt.ctx)
+    if rt.sync_status() != 0:
+        raise RuntimeError("device status set during the timed steps")
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = float(sum(step_ms))
+
+    # ---- stage breakdown (separate pass with per-kernel events; not part of `value`)
+    mla_enable_stage_timing(rt.ctx, True)
+    stage_acc: dict[str, list[float]] = {}
+    for i in range(max(3, min(args.steps, 20))):
+        flush.fill_(float(i))
+        step()
+        for name, ms in mla_stage_times(rt.ctx):
+            stage_acc.setdefault(name, []).append(ms)
+    mla_enable_stage_timing(rt.ctx, False)
+    stages = {k: float(np.mean(v)) for k, v in stage_acc.items()}
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    h_q = torch.empty(q_latent.shape, dtype=torch.bfloat16, pin_memory=True)
+    h_q.copy_(q_latent.cpu())
+    h_sp = torch.empty(start_pos.shape, dtype=torch.int32, pin_memory=True)
+    h_sp.copy_(start_pos.cpu())
+    h_out = torch.empty(out.shape, dtype=torch.bfloat16, pin_memory=True)
+    d_q = torch.empty_like(q_latent)
+    d_sp = torch.empty_like(start_pos)
+    e2e_ms = []
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        d_q.copy_(h_q, non_blocking=True)
+        d_sp.copy_(h_sp, non_blocking=True)
+        if w.mode == "decode":
+            rt.decode(d_q, d_sp, cache, residual=residual, out=out)
+        else:
+            rt.prefill(d_q, w.prefill_start, cache, residual=residual, out=out)
+        h_out.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    h2d = h_q.numel() * 2 + h_sp.numel() * 4
+    d2h = h_out.numel() * 2
+
+    # ---- max over ranks
+    t = torch.tensor([total_ms, float(np.sum(e2e_ms))], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_total = float(t[0]), float(t[1])
+    rt.close()
+    if rank != 0:
+        return None
+
+    peaks = measured_peaks()
+    ms_per_step = total_ms / args.steps
+    units = B * T
+    if w.mode == "decode":
+        value = world * units * args.steps / (total_ms / 1e3)
+        unit = "queries/s"
+        e2e_value = world * units * args.steps / (e2e_total / 1e3)
+    else:
+        value = world * work["flops"] * args.steps / (total_ms / 1e3) / 1e12
+        unit = "TFLOP/s"
+        e2e_value = world * work["flops"] * args.steps / (e2e_total / 1e3) / 1e12
+    attn_ms = stages.get("latent_attention")
+    if w.mode == "decode":
+        achieved = work["attn_bytes"] / (attn_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": None, "kernel": "latent_attention",
+                "algorithmic_bytes_per_launch": work["attn_bytes"],
+                "peak_source": peaks["source"] + " (hbm_gbs, copy burst)"}
+    else:
+        achieved = work["attn_flops"] / (attn_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1),
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops_sustained"], 4), "traffic": None,
+                "kernel": "latent_attention", "algorithmic_flops_per_launch": work["attn_flops"],
+                "peak_source": peaks["source"] + " (bf16_tflops_sustained)"}
+    step_gbs = work["bytes"] / (ms_per_step / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) latents/caches, N(0,1/fan_in) weights)",
+        "config": {"workload": w.name, "batch": B, "tokens": T, "n_heads": H,
+                   "cache_keys_per_step": work["keys"], "q_lora": 1536, "kv_lora": 512,
+                   "rope": 64, "v": 128,
+                   "l2": "flushed before every timed step (256 MiB write, untimed)",
+                   "parallelism": f"replicas x{world} (sequence-sharded, no collective)"},
+        "hbm": {"step_bytes": work["bytes"], "step_gbs": round(step_gbs, 1),
+                "frac_of_peak": round(step_gbs / peaks["hbm_gbs"], 4)},
+        "tflops_step": round(work["flops"] / (ms_per_step / 1e3) / 1e12, 2),
+        "roofline": roof,
+        "stages_ms": {k: round(v, 5) for k, v in stages.items()},
+        "clocks": clk,
+        "e2e": {"value": round(e2e_value, 2), "unit": unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_total / args.steps, 5)},
+        "gpu_launches": launches * args.steps,
+    }
+    return line
+
+
+# ------------------------------------------------------------------------------------------
+# CPU legs: the fp64 oracle on the host cores (bounded sample)
+# ------------------------------------------------------------------------------------------
+def oracle_sample(w, inp, budget_s: float, max_rows: int | None = None) -> dict:
+    """Run the oracle on sequences 0, 1, ... until ~budget_s of CPU time; returns rate."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from mla_cases import oracle_decode, oracle_prefill
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        cores = 1
+    done, t0 = 0, time.perf_counter()
+    if w.mode == "decode":
+        while True:
+            oracle_decode(inp, w, rows=[done % w.batch])
+            done += 1
+            if time.perf_counter() - t0 >= budget_s or (max_rows and done >= max_rows):
+                break
+        el = time.perf_counter() - t0
+        return dict(value=done / el, unit="queries/s", cores=cores,
+                    sample=f"{done} of the {w.batch} sequences' decode (all {w.dims.n_heads} heads) in {el:.1f} s")
+    T = w.tokens
+    work = algorithmic_work(w, inp["start_pos"])
+    per_token = work["flops"] / T
+    while True:
+        oracle_prefill(inp, w, tokens=[(done * 97) % T])
+        done += 1
+        if time.perf_counter() - t0 >= budget_s or (max_rows and done >= max_rows):
+            break
+    el = time.perf_counter() - t0
+    return dict(value=done * per_token / el / 1e12, unit="TFLOP/s", cores=cores,
+                sample=f"{done} of the {T} chunk tokens in {el:.1f} s")
+
+
+def run_reference(args) -> dict:
+    w = workload(args.workload)
+    inp = make_inputs(w, seed=args.seed)
+    per_step = []
+    res = None
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, budget_s=0.0, max_rows=1)
+    for _ in range(args.steps):
+        res = oracle_sample(w, inp, budget_s=args.ref_step_seconds)
+        per_step.append(res["value"])
+    value = float(np.mean(per_step))
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": res["unit"],
+        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "tokens": w.tokens,
+                   "n_heads": w.dims.n_heads},
+        "cpu_baseline": {"kind": "oracle", "cores": res["cores"], "sample": res["sample"],
+                         "value": round(value, 4), "unit": res["unit"]},
+        "e2e": {"value": round(value, 4), "unit": res["unit"], "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="v32_decode")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="budget of the oracle CPU-baseline sample")
+    ap.add_argument("--ref-step-seconds", type=float, default=6.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    line = run_ours(args, rank, world, local_rank)
+    if line is not None:
+        if not args.no_cpu_baseline:
+            w = workload(args.workload)
+            inp = make_inputs(w, seed=args.seed)
+            cb = oracle_sample(w, inp, budget_s=args.cpu_seconds)
+            line["cpu_baseline"] = {"value": round(cb["value"], 4), "unit": cb["unit"],
+                                    "cores": cb["cores"], "kind": "oracle", "sample": cb["sample"]}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,128 @@
+// internal.h — parameter blocks shared between the host launch code (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mla {
+
+typedef __nv_bfloat16 bf16;
+
+// Fixed model dimensions the kernels are built for ("Query heads" page, mla-init excerpt).
+constexpr int kR = 1536;     // q_lora_rank
+constexpr int kC = 512;      // kv_lora_rank
+constexpr int kDn = 128;     // qk_nope_head_dim
+constexpr int kDr = 64;      // qk_rope_head_dim
+constexpr int kDv = 128;     // v_head_dim
+constexpr int kDq = kDn + kDr;        // 192 query features per head
+constexpr int kDk = kC + kDr;         // 576-wide absorbed query / cache row
+constexpr int kHPad = 128;            // heads padded to one 128-row MMA tile
+constexpr int kRopePairs = kDr / 2;   // 32
+
+// ---------------------------------------------------------------------------------------
+// a1: RMSNorm (+ residual) with the rotary table and the per-row key prefix as side outputs
+// ---------------------------------------------------------------------------------------
+struct RmsParams {
+  const bf16* x;            // [rows, dim]
+  bf16* residual;           // [rows, dim] or null (in/out)
+  const float* gamma;       // [dim]
+  bf16* y;                  // [rows, dim]
+  int rows;
+  int dim;
+  float eps;
+  // rotary table (cos, sin) per row and pair; null to skip
+  float2* rope_tab;         // [rows, 32]
+  double rope_log_theta;    // ln(theta)
+  // positions: decode → start_pos_dev[row]; prefill → start_pos + row % T
+  const int32_t* start_pos_dev;
+  int start_pos;
+  int T;
+  int max_seq_len;
+  // key prefix over rows (written by block 0); null to skip
+  long long* row_prefix;    // [rows + 1]
+  int* status;
+};
+
+// ---------------------------------------------------------------------------------------
+// a2/a4/a8: bf16 tensor-core GEMM  D[m, n] = sum_k A[g][m, k] * B[g][n, k]  (both K-major)
+// ---------------------------------------------------------------------------------------
+enum EpiKind : int {
+  kEpiStore = 0,   // out0[n*ld_n0 + g*ld_g0 + m] = bf16(D)
+  kEpiWqbRope = 1, // wq_b: nope rows → q_nope, rope rows → rotated → absorbed-query buffer
+};
+
+struct GemmParams {
+  int M, N, K;
+  int a_row_off;           // row offset of the A tile inside its tensor map
+  int epi;
+  bf16* out0;
+  long long ld_n0, ld_g0;
+  bf16* out1;              // kEpiWqbRope: absorbed-query buffer [rows, 128, 576]
+  const float2* rope_tab;  // [N, 32]
+  int n_heads;
+  int* status;
+};
+
+// ---------------------------------------------------------------------------------------
+// a5–a7: latent flash attention (cluster of two CTAs splits the 576-wide contraction and the
+// 512-wide value dimension), split over keys; rows are query tokens, heads are the MMA M dim.
+// ---------------------------------------------------------------------------------------
+struct AttnParams {
+  const long long* row_prefix;  // [rows + 1] cumulative key counts
+  int rows;
+  int T;                        // prefill tokens per sequence (decode: 1)
+  int n_heads;
+  float scale_log2;             // softmax_scale * log2(e)
+  float scale;                  // softmax_scale
+  int min_keys_per_pair;
+  bf16* o_lat;                  // [rows, H, 512] bf16 (rows attended by one pair only)
+  float* lse_out;               // [rows, H] or null
+  float* logits;                // [B, H, max_seq_len] or null (decode debug)
+  int max_seq_len;
+  float* part_o;                // [pairs, 2, 128, 512] fp32 normalised partial outputs
+  float* part_lse;              // [pairs, 2, 128]
+  int* status;
+};
+
+struct CombineParams {
+  const long long* row_prefix;
+  int rows;
+  int n_heads;
+  int n_pairs;                  // pairs the attention kernel launched
+  int min_keys_per_pair;
+  const float* part_o;
+  const float* part_lse;
+  bf16* o_lat;
+  float* lse_out;
+};
+
+// Launchers (defined next to their kernels).
+cudaError_t launch_rmsnorm(const RmsParams& p, cudaStream_t s);
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+                        int batches, cudaStream_t s);
+cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tpe,
+                             const AttnParams& p, int n_pairs, cudaStream_t s);
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
+cudaError_t launch_transpose_uk(const bf16* wkv_b, bf16* w_ukt, int n_heads, cudaStream_t s);
+cudaError_t gemm_prepare();        // one-time per-device attribute set-up
+cudaError_t attention_prepare();
+
+// Token-tile width the GEMM launcher picks for N token rows (the B operand's TMA box height).
+inline int gemm_bn(int n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : 256; }
+
+// Number of cluster pairs the attention kernel uses on this device (SMs / 2).
+int attention_pairs();
+
+// Pair partition of the flattened key range, shared by the attention and combine kernels.
+__host__ __device__ inline int active_pairs(long long total_keys, int launched, int min_keys) {
+  long long want = (total_keys + min_keys - 1) / min_keys;
+  if (want < 1) want = 1;
+  return want < launched ? static_cast<int>(want) : launched;
+}
+__host__ __device__ inline long long pair_begin(long long total_keys, int pairs, int p) {
+  return total_keys * p / pairs;
+}
+
+}  // namespace mla

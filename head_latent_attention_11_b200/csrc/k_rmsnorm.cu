@@ -1,0 +1,143 @@
+// k_rmsnorm.cu — a1: q_norm RMSNorm with optional fused residual add.
+//
+// "DeepSeek-V3.2-Exp · Attention update", rmsnorm excerpt: in fp32, u = x (+ residual); the new
+// residual is u cast back to the input type; y = gain * u * rsqrt(mean(u^2) + eps), cast back.
+// "DeepSeek V4.1 · Query RMSNorm" gives the same formula.
+//
+// One warp per row; each lane holds dim/32 values in registers (16-byte bf16 vector loads and
+// stores, fully coalesced), the sum of squares is reduced with warp shuffles.  The decode/prefill
+// chain also uses this kernel to emit two small side outputs so that no extra launch is needed:
+//   * the rotary table (cos, sin) of each row's position for the 32 interleaved pairs
+//     ("Query heads" page: R [T positions, 32 pairs]), angles evaluated in double precision;
+//   * the cumulative key count of the rows (block 0), used by the attention and combine kernels
+//     to split the flattened key range evenly across SM pairs.
+#include "internal.h"
+#include "tc100.cuh"
+
+namespace mla {
+
+__device__ __forceinline__ int row_position(const RmsParams& p, int row, bool* bad) {
+  int pos;
+  if (p.start_pos_dev) {
+    pos = p.start_pos_dev[row];
+  } else {
+    pos = p.start_pos + row % p.T;
+  }
+  if (pos < 0 || pos >= p.max_seq_len) {
+    *bad = true;
+    pos = pos < 0 ? 0 : p.max_seq_len - 1;
+  }
+  return pos;
+}
+
+__device__ void key_prefix_block(const RmsParams& p) {
+  // 128 threads; thread t owns rows [t*chunk, (t+1)*chunk)
+  __shared__ long long part[128];
+  const int t = threadIdx.x;
+  const int chunk = (p.rows + 127) / 128;
+  const int r0 = min(p.rows, t * chunk), r1 = min(p.rows, r0 + chunk);
+  long long local = 0;
+  bool bad = false;
+  for (int r = r0; r < r1; ++r) local += row_position(p, r, &bad) + 1;
+  part[t] = local;
+  __syncthreads();
+  if (t == 0) {
+    long long acc = 0;
+    for (int i = 0; i < 128; ++i) {
+      long long v = part[i];
+      part[i] = acc;
+      acc += v;
+    }
+  }
+  __syncthreads();
+  long long acc = part[t];
+  if (t == 0) p.row_prefix[0] = 0;
+  for (int r = r0; r < r1; ++r) {
+    acc += row_position(p, r, &bad) + 1;
+    p.row_prefix[r + 1] = acc;
+  }
+  if (bad) atomicCAS(p.status, kDevOk, kDevBadArg);
+}
+
+template <int NCH>
+__global__ void __launch_bounds__(128) rmsnorm_kernel(const RmsParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 4 + warp;
+  if (row < p.rows) {
+    const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(row) * p.dim);
+    uint4* rr = p.residual ? reinterpret_cast<uint4*>(p.residual + static_cast<size_t>(row) * p.dim)
+                           : nullptr;
+    float u[NCH][8];
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int idx = lane + 32 * c;
+      uint4 xv = xr[idx];
+      const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(&xv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) u[c][i] = __bfloat162float(xb[i]);
+      if (rr) {
+        uint4 rv = rr[idx];
+        const __nv_bfloat16* rb = reinterpret_cast<const __nv_bfloat16*>(&rv);
+        uint4 ov;
+        uint32_t* o32 = reinterpret_cast<uint32_t*>(&ov);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) u[c][i] += __bfloat162float(rb[i]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o32[i] = pack_bf16x2(u[c][2 * i], u[c][2 * i + 1]);
+        rr[idx] = ov;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss = fmaf(u[c][i], u[c][i], ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = rsqrtf(ss / static_cast<float>(p.dim) + p.eps);
+    uint4* yr = reinterpret_cast<uint4*>(p.y + static_cast<size_t>(row) * p.dim);
+    const float4* g4 = reinterpret_cast<const float4*>(p.gamma);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int idx = lane + 32 * c;
+      const float4 ga = g4[2 * idx], gb = g4[2 * idx + 1];
+      const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+      uint4 ov;
+      uint32_t* o32 = reinterpret_cast<uint32_t*>(&ov);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o32[i] = pack_bf16x2(g[2 * i] * (u[c][2 * i] * inv), g[2 * i + 1] * (u[c][2 * i + 1] * inv));
+      yr[idx] = ov;
+    }
+    if (p.rope_tab) {
+      bool bad = false;
+      const int pos = row_position(p, row, &bad);
+      // theta_i = theta^(-2i/64); lane i owns pair i
+      const double inv_freq = exp(-2.0 * static_cast<double>(lane) / kDr * p.rope_log_theta);
+      double sn, cs;
+      sincos(static_cast<double>(pos) * inv_freq, &sn, &cs);
+      p.rope_tab[static_cast<size_t>(row) * kRopePairs + lane] =
+          make_float2(static_cast<float>(cs), static_cast<float>(sn));
+    }
+  }
+  if (blockIdx.x == 0 && p.row_prefix) key_prefix_block(p);
+}
+
+cudaError_t launch_rmsnorm(const RmsParams& p, cudaStream_t s) {
+  const int nch = p.dim / 256;
+  dim3 grid((p.rows + 3) / 4), block(128);
+  switch (nch) {
+#define MLA_RMS_CASE(n) \
+  case n:               \
+    rmsnorm_kernel<n><<<grid, block, 0, s>>>(p); \
+    break;
+    MLA_RMS_CASE(1) MLA_RMS_CASE(2) MLA_RMS_CASE(3) MLA_RMS_CASE(4) MLA_RMS_CASE(5)
+    MLA_RMS_CASE(6) MLA_RMS_CASE(7) MLA_RMS_CASE(8) MLA_RMS_CASE(9) MLA_RMS_CASE(10)
+    MLA_RMS_CASE(11) MLA_RMS_CASE(12) MLA_RMS_CASE(13) MLA_RMS_CASE(14) MLA_RMS_CASE(15)
+    MLA_RMS_CASE(16)
+#undef MLA_RMS_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -162,7 +162,7 @@ def make_inputs(w: Workload, seed: int = 0, tail: str = "zero", max_t: int | Non
     start_pos = _start_positions(w, np.random.default_rng(s_pos))
     n_keys = start_pos.astype(np.int64) + w.tokens           # keys of the last query of each row
     if max_t is None:
-        max_t = int(n_keys.max())
+        max_t = max(64, int(n_keys.max()))   # the library wants at least 64 cache rows
     if max_t < int(n_keys.max()):
         raise ValueError("max_t smaller than the longest sequence")
 

@@ -5,9 +5,10 @@ benchmark may import this module.  The library's GPU path never calls it and sha
 with it; this file imports nothing but numpy.
 
 Every function follows one passage of the source pages and is written as the plain definition,
-in float64, with no intermediate rounding (the pages round to bf16 after each Linear/einsum; the
-GPU path rounds at similar points and the parity tolerance absorbs it).  Library primitives used
-as steps: numpy ``matmul``/``einsum`` (contractions), ``exp``/``log``/``sqrt``/``sin``/``cos``.
+in float64.  By default nothing is rounded in between (the pages round to bf16 after each
+Linear/einsum; the GPU path rounds at similar points and the parity tolerance absorbs it); see the
+precision modes below.  Library primitives used as steps: numpy ``matmul``/``einsum``
+(contractions), ``exp``/``log``/``sqrt``/``sin``/``cos``/``frexp``/``rint``.
 
 Source pages (cited by title and section):
   [QRMS]  DeepSeek V4.1 · Query RMSNorm — formula block and the ``RMSNorm`` excerpt.
@@ -27,16 +28,34 @@ Readings where the pages are silent or garbled (each also listed in the design n
   * Decode query sits at position start_pos and sees keys 0..start_pos; a prefill query t sees
     keys 0..start_pos+t.
   * softmax_scale = qk_head_dim^-0.5 (the YaRN mscale branch of [QH] mla-init is off).
+
+Precision modes of ``decode`` / ``prefill``:
+  * ``query_precision="exact"`` (default): every step in float64, no rounding.
+  * ``query_precision="bf16"``: the query side is rounded to bfloat16 where the pages' tensors are
+    bfloat16 — the RMSNorm output (``.to(dtype)``, [AU] rmsnorm), the wq_b output (a bf16
+    Linear, [QH] mla-queries), the rotated q_pe (``apply_rotary_emb`` returns the input dtype,
+    [QH] mla-queries) and the absorbed q_nope (einsum of bf16 tensors, [AU] mla-decode).  Scores,
+    softmax and everything after stay float64 (the fp32 softmax of the method).  This is the
+    reference for the softmax probabilities, whose 1e-3 bound is tighter than the effect of those
+    four roundings.
 """
 from __future__ import annotations
 
 import numpy as np
 
 __all__ = [
-    "rmsnorm", "rope_frequencies", "apply_rope_interleaved", "query_heads", "absorb_w_uk",
+    "round_bf16", "rmsnorm", "rope_frequencies", "apply_rope_interleaved", "query_heads", "absorb_w_uk",
     "latent_scores", "softmax_fp", "latent_weighted_sum", "expand_w_uv", "decode", "prefill",
     "nonabsorbed_attention", "split_wkv_b", "split_wq_b",
 ]
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 value (8 significant bits, ties to even),
+    returned as float64.  Done directly from float64 (no detour through float32)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                       # x = m * 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.rint(m * 256.0), e - 8)
 
 
 # ------------------------------------------------------------------------------------------
@@ -153,12 +172,22 @@ def _attend_row(q_lat_h, q_pe_h, kv, pe, scale, w_uv, want_logits=False):
     return out, lse, (s if want_logits else None), o_lat
 
 
-def _front(q_latent_rows, residual_rows, gamma, wq_b, wkv_b, dims, pos, theta, eps):
+def _front(q_latent_rows, residual_rows, gamma, wq_b, wkv_b, dims, pos, theta, eps,
+           query_precision="exact"):
     H, nope, rope, v = dims["n_heads"], dims["nope"], dims["rope"], dims["v"]
-    y, res = rmsnorm(q_latent_rows, gamma, eps, residual_rows)
-    q_nope, q_pe = query_heads(y, wq_b, H, nope, rope, pos, theta)
     w_uk, w_uv = split_wkv_b(wkv_b, H, nope, v)
-    q_lat = absorb_w_uk(q_nope, w_uk)
+    y, res = rmsnorm(q_latent_rows, gamma, eps, residual_rows)
+    if query_precision == "exact":
+        q_nope, q_pe = query_heads(y, wq_b, H, nope, rope, pos, theta)
+        q_lat = absorb_w_uk(q_nope, w_uk)
+    elif query_precision == "bf16":
+        y = round_bf16(y)
+        q = round_bf16(y @ np.asarray(wq_b, dtype=np.float64).T).reshape(y.shape[0], H, nope + rope)
+        q_nope = q[..., :nope]
+        q_pe = round_bf16(apply_rope_interleaved(q[..., nope:], np.asarray(pos)[:, None], theta))
+        q_lat = round_bf16(absorb_w_uk(q_nope, w_uk))
+    else:
+        raise ValueError(query_precision)
     return y, res, q_nope, q_pe, q_lat, w_uv
 
 
@@ -168,7 +197,7 @@ def _dims(n_heads, nope=128, rope=64, v=128):
 
 def decode(q_latent, gamma, wq_b, wkv_b, cache, start_pos, n_heads, *, residual=None,
            kv_lora=512, nope=128, rope=64, v=128, theta=10000.0, eps=1e-6, scale=None,
-           rows=None, want_logits=False, want_intermediates=False):
+           rows=None, want_logits=False, want_intermediates=False, query_precision="exact"):
     """Absorbed decode ([AU] mla-decode with the index mask keeping every key).
 
     ``q_latent`` [B, q_lora]; ``cache`` [B, max_t, kv_lora+rope] (packed latents ‖ pe key);
@@ -184,7 +213,7 @@ def decode(q_latent, gamma, wq_b, wkv_b, cache, start_pos, n_heads, *, residual=
     res_in = None if residual is None else np.asarray(residual, np.float64)[rows]
     pos = np.asarray(start_pos)[rows].astype(np.int64)
     y, res, q_nope, q_pe, q_lat, w_uv = _front(q_latent, res_in, gamma, wq_b, wkv_b, dims,
-                                                pos, theta, eps)
+                                                pos, theta, eps, query_precision)
     outs, lses, logits, olats = [], [], [], []
     for i, b in enumerate(rows):
         n = int(pos[i]) + 1
@@ -206,7 +235,7 @@ def decode(q_latent, gamma, wq_b, wkv_b, cache, start_pos, n_heads, *, residual=
 
 def prefill(q_latent, gamma, wq_b, wkv_b, cache, start_pos, n_heads, *, residual=None,
             kv_lora=512, nope=128, rope=64, v=128, theta=10000.0, eps=1e-6, scale=None,
-            batch_rows=None, tokens=None, want_intermediates=False):
+            batch_rows=None, tokens=None, want_intermediates=False, query_precision="exact"):
     """Absorbed attention for a chunk of T new tokens after ``start_pos`` (int) cached positions.
 
     Query t of sequence b is at position start_pos + t and sees keys 0..start_pos+t (causal;
@@ -229,7 +258,7 @@ def prefill(q_latent, gamma, wq_b, wkv_b, cache, start_pos, n_heads, *, residual
         rs = None if residual is None else np.asarray(residual, np.float64)[b, tokens]
         pos = int(start_pos) + tokens.astype(np.int64)
         y, res, q_nope, q_pe, q_lat, w_uv = _front(xs, rs, gamma, wq_b, wkv_b, dims, pos,
-                                                    theta, eps)
+                                                    theta, eps, query_precision)
         for ti in range(len(tokens)):
             n = int(pos[ti]) + 1
             kv = np.asarray(cache[b, :n, :kv_lora], np.float64)

@@ -1,0 +1,88 @@
+"""Helpers shared by the GPU parity tests: move seeded inputs to the device, run the library
+through the C ABI, run the oracle on the same bf16 values and compare within the stated bounds.
+
+Tolerances (stated for the path): bf16 outputs |err| <= 1e-2 * max|ref| + 1e-3; softmax
+probabilities within 1e-3 absolute.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from mla_synth import bf16_bits_to_f64, make_inputs, workload
+
+REL_TOL = 1e-2
+ABS_TOL = 1e-3
+PROB_TOL = 1e-3
+
+
+def assert_close_bf16(got: np.ndarray, ref: np.ndarray, what: str, rel=REL_TOL, abs_=ABS_TOL):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, f"{what}: shape {got.shape} vs {ref.shape}"
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    bound = rel * float(np.max(np.abs(ref))) + abs_
+    err = float(np.max(np.abs(got - ref)))
+    assert err <= bound, f"{what}: max|err| {err:.3e} > bound {bound:.3e}"
+    return err, bound
+
+
+def to_device(inp: dict, device="cuda"):
+    import torch
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+    d = {
+        "q_latent": bf16(inp["q_latent"]),
+        "residual": None if inp["residual"] is None else bf16(inp["residual"]),
+        "gamma": torch.from_numpy(inp["gamma"]).to(device),
+        "wq_b": bf16(inp["wq_b"]),
+        "wkv_b": bf16(inp["wkv_b"]),
+        "cache": bf16(inp["cache"]),
+        "start_pos": torch.from_numpy(inp["start_pos"].astype(np.int32)).to(device),
+    }
+    return d
+
+
+def bf16_to_np(t) -> np.ndarray:
+    import torch
+    return t.detach().to("cpu").view(torch.int16).numpy().view(np.uint16)
+
+
+def f64(t) -> np.ndarray:
+    return bf16_bits_to_f64(bf16_to_np(t))
+
+
+def oracle_decode(inp: dict, w, rows=None, **kw):
+    d = w.dims
+    return oracle.decode(
+        bf16_bits_to_f64(inp["q_latent"][:, 0]), inp["gamma"].astype(np.float64),
+        bf16_bits_to_f64(inp["wq_b"]), bf16_bits_to_f64(inp["wkv_b"]), _CacheView(inp["cache"]),
+        inp["start_pos"], d.n_heads,
+        residual=None if inp["residual"] is None else bf16_bits_to_f64(inp["residual"][:, 0]),
+        theta=w.rope_theta, eps=w.rms_eps, rows=rows, **kw)
+
+
+def oracle_prefill(inp: dict, w, tokens=None, **kw):
+    d = w.dims
+    return oracle.prefill(
+        bf16_bits_to_f64(inp["q_latent"]), inp["gamma"].astype(np.float64),
+        bf16_bits_to_f64(inp["wq_b"]), bf16_bits_to_f64(inp["wkv_b"]), _CacheView(inp["cache"]),
+        int(inp["start_pos"][0]), d.n_heads,
+        residual=None if inp["residual"] is None else bf16_bits_to_f64(inp["residual"]),
+        theta=w.rope_theta, eps=w.rms_eps, tokens=tokens, **kw)
+
+
+class _CacheView:
+    """Widens rows of the bf16 cache to float64 lazily (indexing [b, :n, cols])."""
+
+    def __init__(self, bits: np.ndarray):
+        self.bits = bits
+
+    def __getitem__(self, idx):
+        return bf16_bits_to_f64(self.bits[idx])
+
+
+__all__ = ["assert_close_bf16", "to_device", "bf16_to_np", "f64", "oracle_decode",
+           "oracle_prefill", "make_inputs", "workload", "REL_TOL", "ABS_TOL", "PROB_TOL"]

@@ -323,6 +323,38 @@ def test_brute_force_tiny(seed):
 
 
 # ------------------------------------------------------------------------------------------
+# bf16 rounding of the oracle's "bf16" precision mode
+# ------------------------------------------------------------------------------------------
+def test_round_bf16_matches_torch_and_ties_to_even():
+    import torch
+    rng = np.random.default_rng(14)
+    a = (rng.standard_normal(200000) * np.exp(rng.uniform(-20, 20, 200000))).astype(np.float32)
+    ref = torch.from_numpy(a).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.round_bf16(a.astype(np.float64)), ref)
+    # halfway cases: 1 + 2^-8 lies between 1 and 1 + 2^-7 -> even (1.0); 1 + 3*2^-8 -> 1 + 2^-6
+    assert oracle.round_bf16(np.array(1 + 2.0 ** -8)) == 1.0
+    assert oracle.round_bf16(np.array(1 + 3 * 2.0 ** -8)) == 1 + 2.0 ** -6
+    # just above a tie (not representable in fp32) must round up, directly from float64
+    assert oracle.round_bf16(np.array(1 + 2.0 ** -8 + 2.0 ** -40)) == 1 + 2.0 ** -7
+    x = rng.standard_normal(1000)
+    np.testing.assert_array_equal(oracle.round_bf16(oracle.round_bf16(x)), oracle.round_bf16(x))
+
+
+def test_bf16_query_mode_stays_close_to_exact():
+    """The pages' bf16 query roundings move the output by far less than the parity bound."""
+    w = workload("tiny_decode")
+    inp = make_inputs(w, seed=2)
+    args = (bf16_bits_to_f64(inp["q_latent"][:, 0]), inp["gamma"].astype(np.float64),
+            bf16_bits_to_f64(inp["wq_b"]), bf16_bits_to_f64(inp["wkv_b"]),
+            bf16_bits_to_f64(inp["cache"]), inp["start_pos"], 16)
+    ex = oracle.decode(*args, want_intermediates=True)
+    bq = oracle.decode(*args, want_intermediates=True, query_precision="bf16")
+    assert np.max(np.abs(bq["out"] - ex["out"])) < 5e-3 * np.max(np.abs(ex["out"]))
+    np.testing.assert_array_equal(bq["q_lat"], oracle.round_bf16(bq["q_lat"]))
+    assert not np.array_equal(bq["q_lat"], ex["q_lat"])
+
+
+# ------------------------------------------------------------------------------------------
 # Input generator
 # ------------------------------------------------------------------------------------------
 def test_bf16_rounding_matches_torch():
@@ -344,7 +376,7 @@ def test_generator_is_seeded_and_shaped():
     assert not np.array_equal(a["cache"], c["cache"])
     assert a["q_latent"].shape == (2, 1, 1536)
     assert a["wq_b"].shape == (16 * 192, 1536) and a["wkv_b"].shape == (16 * 256, 512)
-    assert a["cache"].shape == (2, 129, 576) and list(a["start_pos"]) == [128, 128]
+    assert a["cache"].shape == (2, 129, 576)  # max_t = L + 1 and list(a["start_pos"]) == [128, 128]
     wq = bf16_bits_to_f64(a["wq_b"])
     assert abs(wq.std() * math.sqrt(1536) - 1) < 0.01
     wr = workload("ragged_decode", batch=8)
