@@ -194,17 +194,15 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   int launches = 0;
 
   // per-call tensor maps
-  CUtensorMap tm_y, tm_qn, tm_olat, tm_q, tm_kv, tm_pe;
+  CUtensorMap tm_y, tm_qn, tm_olat, tm_kv, tm_pe;
   const uint64_t rws = static_cast<uint64_t>(rows);
   if (!make_map(&tm_y, c->y(), kR, 1, rws, kR * 2, kR * 2, 64, 1, bn) ||
       !make_map(&tm_qn, c->q_nope(), kDn, H, rws, kDn * 2, static_cast<uint64_t>(H) * kDn * 2, 64,
                 1, bn) ||
       !make_map(&tm_olat, c->o_lat(), kC, H, rws, kC * 2, static_cast<uint64_t>(H) * kC * 2, 64, 1,
                 bn) ||
-      !make_map(&tm_q, c->qabs(), kDk, kHPad, rws, kDk * 2, static_cast<uint64_t>(kHPad) * kDk * 2,
-                64, 128, 1) ||
-      !make_map(&tm_kv, kv, kC, c->cfg.max_seq_len, B, kv_st * 2, kv_sb * 2, 64, 64, 1) ||
-      !make_map(&tm_pe, pe, kDr, c->cfg.max_seq_len, B, pe_st * 2, pe_sb * 2, 64, 64, 1))
+      !make_map(&tm_kv, kv, kC, c->cfg.max_seq_len, B, kv_st * 2, kv_sb * 2, 64, kAttnKeysPerTile, 1) ||
+      !make_map(&tm_pe, pe, kDr, c->cfg.max_seq_len, B, pe_st * 2, pe_sb * 2, 64, kAttnKeysPerTile, 1))
     return MLA_ERR_INVALID_ARG;
 
   // 1. q_norm (+ residual), rotary table, key prefix
@@ -262,6 +260,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   // 4. latent attention
   AttnParams ap{};
   ap.row_prefix = c->prefix();
+  ap.qabs = c->qabs();
   ap.rows = rows;
   ap.T = T;
   ap.n_heads = H;
@@ -276,7 +275,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   ap.part_lse = c->part_lse();
   ap.status = c->status();
   clk.mark("latent_attention");
-  MLA_TRY(launch_attention(tm_q, tm_kv, tm_pe, ap, c->n_pairs, s));
+  MLA_TRY(launch_attention(tm_kv, tm_pe, ap, c->n_pairs, s));
   ++launches;
 
   // 5. combine rows cut between pairs

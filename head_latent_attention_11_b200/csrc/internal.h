@@ -20,6 +20,7 @@ constexpr int kDq = kDn + kDr;        // 192 query features per head
 constexpr int kDk = kC + kDr;         // 576-wide absorbed query / cache row
 constexpr int kHPad = 128;            // heads padded to one 128-row MMA tile
 constexpr int kRopePairs = kDr / 2;   // 32
+constexpr int kAttnKeysPerTile = 32;  // cache rows per attention tile (TMA box height)
 
 // ---------------------------------------------------------------------------------------
 // a1: RMSNorm (+ residual) with the rotary table and the per-row key prefix as side outputs
@@ -71,6 +72,7 @@ struct GemmParams {
 // ---------------------------------------------------------------------------------------
 struct AttnParams {
   const long long* row_prefix;  // [rows + 1] cumulative key counts
+  const bf16* qabs;             // [rows, 128, 576] absorbed query (q_lat ‖ q_pe), heads padded
   int rows;
   int T;                        // prefill tokens per sequence (decode: 1)
   int n_heads;
@@ -102,8 +104,8 @@ struct CombineParams {
 cudaError_t launch_rmsnorm(const RmsParams& p, cudaStream_t s);
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                         int batches, cudaStream_t s);
-cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tpe,
-                             const AttnParams& p, int n_pairs, cudaStream_t s);
+cudaError_t launch_attention(const CUtensorMap& tkv, const CUtensorMap& tpe, const AttnParams& p,
+                             int n_pairs, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 cudaError_t launch_transpose_uk(const bf16* wkv_b, bf16* w_ukt, int n_heads, cudaStream_t s);
 cudaError_t gemm_prepare();        // one-time per-device attribute set-up

@@ -8,23 +8,33 @@
 //
 // Design (B200):
 //   * One query row (one token of one sequence) at a time; its heads form the MMA M dimension
-//     (128 rows, heads beyond H are zero rows), so QK^T and P·V are dense 128-row tcgen05 MMAs.
+//     (128 rows; heads beyond H are zero rows), so QK^T and P·V are dense 128-row tcgen05 MMAs.
 //   * A cluster of TWO CTAs (one SM each) handles a row.  CTA 0 owns the latent columns
-//     [0, 256), CTA 1 owns [256, 512) plus the 64 rotary columns.  Each CTA loads only its
-//     columns of every cache tile (so the 576-wide cache row is read from HBM once), computes a
-//     partial score tile over its columns, and the two partials are exchanged through
-//     distributed shared memory; both CTAs then hold identical full scores and run the identical
-//     online softmax.  Each CTA accumulates the value half it owns: O[128 x 256] fp32 in TMEM
-//     (256 columns), plus two 64-column score buffers.
-//   * Keys are streamed in tiles of 64 by TMA (128-byte swizzle, evict-first), two stages deep.
+//     [0, 256); CTA 1 owns [256, 512) and the 64 rotary columns.  Each CTA streams only its
+//     columns of every cache tile (the 576-wide cache row crosses HBM once), computes a partial
+//     score tile over them and sends it to the peer through distributed shared memory; both CTAs
+//     then hold identical full scores and run the identical online softmax.  Each CTA
+//     accumulates the value half it owns, O[128 x 256] fp32 in TMEM.
+//   * The CTA's half of the absorbed query lives in TMEM and is the A operand of the score MMA;
+//     the probabilities P (bf16) overwrite the score tile in TMEM and are the A operand of the
+//     P·V MMA.  Shared memory then holds only the cache ring (32-key tiles, 8 stages deep, TMA
+//     with 128-byte swizzle, evict-first) and the two exchange slots.
+//     TMEM columns: O [0,256) | query half [256,416) | three 32-column score/P buffers [416,512).
+//     With three buffers the score MMA of tile g only waits for P·V of tile g-3, so the tensor
+//     core runs two tiles ahead of the softmax.
+//   * The score exchange uses st.async: the partial scores land in the peer's shared memory and
+//     complete a transaction count on the peer's barrier, so the sender never stalls.  It is also
+//     software-pipelined: a thread sends tile g's partial scores, then finishes tile g-1 (whose
+//     partner half has arrived meanwhile).
 //   * The flattened key range of all rows is split evenly over the cluster pairs (split-K over
 //     keys, also across row boundaries); a row cut between pairs leaves normalised partials
 //     (O/l, lse) for the combine kernel, an uncut row is written as bf16 o_lat directly.
 //   * Online softmax in exp2 domain with lazy rescaling: the running max is only raised (and O
 //     in TMEM rescaled) when a tile's max exceeds it by more than 8 (factor 256), which keeps the
 //     rescale off the common path while the result stays exact.
-//   * Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-5 softmax and
-//     epilogue (thread = head row = TMEM lane).
+//   * Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-5 query loader,
+//     softmax and epilogue (thread = head row = TMEM lane).
+//   * Every wait is bounded (see tc100.cuh); a stuck pipeline records a status and ends.
 #include "internal.h"
 #include "tc100.cuh"
 
@@ -32,41 +42,38 @@ namespace mla {
 
 namespace {
 
-constexpr int kNK = 64;                    // keys per tile
-constexpr int kStages = 2;                 // cache tile ring depth
-constexpr int kSlabKV = kNK * 128;         // 8 KB: 64 columns x 64 keys, bf16
-constexpr int kSlabQ = 128 * 128;          // 16 KB: 64 columns x 128 heads, bf16
+constexpr int kNK = kAttnKeysPerTile;      // keys per tile
+constexpr int kStages = 8;                 // cache tile ring depth
+constexpr int kSlabKV = kNK * 128;         // 4 KB: 64 columns x 32 keys, bf16
 constexpr int kMaxSlabs = 5;               // rank 1: 4 latent slabs + 1 rotary slab
 constexpr int kStageBytes = kMaxSlabs * kSlabKV;
-constexpr int kPBytes = 128 * kNK * 2;     // 16 KB
-constexpr int kXBytes = 128 * kNK * 4;     // 32 KB
+constexpr int kXSlot = 128 * kNK * 4;      // 16 KB: one partial score tile, fp32
 
-constexpr int kOffQ = 0;
-constexpr int kOffKV = kOffQ + kMaxSlabs * kSlabQ;        // 80 KB
-constexpr int kOffP = kOffKV + kStages * kStageBytes;     // 160 KB
-constexpr int kOffX = kOffP + 2 * kPBytes;                // 192 KB
-constexpr int kOffBar = kOffX + kXBytes;                  // 224 KB
-constexpr int kAttnSmem = kOffBar + 256 + 1024;
+constexpr int kOffKV = 0;
+constexpr int kOffX = kOffKV + kStages * kStageBytes;     // 160 KB
+constexpr int kOffBar = kOffX + 2 * kXSlot;               // 192 KB
+constexpr int kAttnSmem = kOffBar + 512 + 1024;
 
 constexpr int kTmemCols = 512;
-constexpr uint32_t kTmemO = 0;             // columns [0, 256)
-constexpr uint32_t kTmemS = 256;           // two 64-column score buffers
+constexpr uint32_t kTmemO = 0;             // [0, 256)
+constexpr uint32_t kTmemQ = 256;           // [256, 416): up to 320 bf16 K-columns
+constexpr uint32_t kTmemS = 416;           // three 32-column score / probability buffers
+constexpr int kNS = 3;
 
 constexpr int kThreads = 192;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct Bars {
-  uint64_t q_full, q_empty;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], pv_done[2];
+  uint64_t q_full, q_empty;
+  uint64_t s_full[kNS], p_full[kNS], pv_done[kNS];
   uint64_t o_empty;
-  uint64_t x_full, x_empty;
+  uint64_t x_full[2], x_empty[2];
   uint64_t drain;
   uint32_t tmem_slot;
   int abort_flag;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block");
+static_assert(sizeof(Bars) <= 512, "barrier block");
 
 // Row containing flattened key e: largest r with prefix[r] <= e.
 __device__ __forceinline__ int row_of_key(const long long* prefix, int rows, long long e) {
@@ -92,7 +99,6 @@ struct PieceIter {
     e1 = e;
     r = row_of_key(pf, nrows, b);
   }
-  // Fills the current piece; false when the range is exhausted.
   __device__ bool get(int& row, int& k0, int& k1, int& nkeys_row, bool& first_row) const {
     if (r >= rows) return false;
     const long long R0 = __ldg(prefix + r), R1 = __ldg(prefix + r + 1);
@@ -107,17 +113,19 @@ struct PieceIter {
   __device__ void next() { ++r; }
 };
 
+__device__ __forceinline__ uint32_t xbuf_off(int slot, int h, int c) {
+  // row h of a slot holds 32 floats = 8 chunks of 16 B; chunk c is stored at (c + h) & 7
+  return static_cast<uint32_t>(slot * kXSlot + h * 128 + (((c + h) & 7) << 4));
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    latent_attention_kernel(const __grid_constant__ CUtensorMap tmQ,
-                            const __grid_constant__ CUtensorMap tmKV,
+    latent_attention_kernel(const __grid_constant__ CUtensorMap tmKV,
                             const __grid_constant__ CUtensorMap tmPE, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem + kOffQ;
   uint8_t* sKV = smem + kOffKV;
-  uint8_t* sP = smem + kOffP;
-  float* sX = reinterpret_cast<float*>(smem + kOffX);
+  uint8_t* sX = smem + kOffX;
   Bars* bar = reinterpret_cast<Bars*>(smem + kOffBar);
 
   const uint32_t rank = cluster_ctarank();
@@ -130,30 +138,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const long long e0 = pair_begin(total, pairs, pair), e1 = pair_begin(total, pairs, pair + 1);
 
   const int warp = static_cast<int>(warp_id());
-  const int nslabs = rank == 0 ? 4 : 5;           // column slabs this CTA owns
-  const int col0 = rank == 0 ? 0 : 256;           // first latent column
+  const int nslabs = rank == 0 ? 4 : 5;           // 64-column slabs this CTA owns
+  const int col0 = rank == 0 ? 0 : 256;           // first cache / query column it owns
   Guard guard{reinterpret_cast<volatile int*>(&bar->abort_flag), p.status};
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar->q_full, 1);
-    mbar_init(&bar->q_empty, 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&bar->kv_full[i], 1);
       mbar_init(&bar->kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(&bar->q_full, 128);
+    mbar_init(&bar->q_empty, 1);
+    for (int i = 0; i < kNS; ++i) {
       mbar_init(&bar->s_full[i], 1);
-      mbar_init(&bar->s_empty[i], 128);
       mbar_init(&bar->p_full[i], 128);
       mbar_init(&bar->pv_done[i], 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar->x_full[i], 1);     // receiver's expect_tx arrival + the peer's bytes
+      mbar_init(&bar->x_empty[i], 4);    // one arrival per softmax warp of the peer
+    }
     mbar_init(&bar->o_empty, 128);
-    mbar_init(&bar->x_full, 128);
-    mbar_init(&bar->x_empty, 128);
     mbar_init(&bar->drain, 1);
     bar->abort_flag = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmKV);
     tma_prefetch_desc(&tmPE);
   }
@@ -171,20 +179,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- TMA producer
     if (elect_one()) {
       const uint64_t pol = policy_evict_first();
-      int g = 0, piece = 0;
-      int last_q = -1;
-      int last_tile[kStages] = {-1, -1};
+      int g = 0;
+      int last_tile[kStages];
+      for (int s = 0; s < kStages; ++s) last_tile[s] = -1;
       int row, k0, k1, nrow;
       bool first_row;
-      while (!guard.aborted() && it.get(row, k0, k1, nrow, first_row)) {
+      bool ok = true;
+      while (ok && it.get(row, k0, k1, nrow, first_row)) {
         const int b = row / p.T;
-        if (piece > 0 && !mbar_wait(&bar->q_empty, (piece - 1) & 1, guard)) break;
-        mbar_arrive_expect_tx(&bar->q_full, nslabs * kSlabQ);
-        for (int i = 0; i < nslabs; ++i)
-          tma_load_3d(sQ + i * kSlabQ, &tmQ, &bar->q_full, col0 + 64 * i, 0, row);
-        last_q = piece;
         const int ntiles = (k1 - k0 + kNK - 1) / kNK;
-        bool ok = true;
         for (int j = 0; j < ntiles; ++j, ++g) {
           const int s = g % kStages;
           if (g >= kStages && !mbar_wait(&bar->kv_empty[s], ((g / kStages) - 1) & 1, guard)) {
@@ -200,14 +203,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (rank == 1) tma_load_3d_hint(dst + 4 * kSlabKV, &tmPE, fb, 0, key, b, pol);
           last_tile[s] = g;
         }
-        if (!ok) break;
-        ++piece;
         it.next();
       }
       if (guard.aborted()) {
         int dummy = 0;
         Guard drain{reinterpret_cast<volatile int*>(&dummy), p.status};
-        if (last_q >= 0) mbar_wait(&bar->q_full, last_q & 1, drain);
         for (int s = 0; s < kStages; ++s)
           if (last_tile[s] >= 0) mbar_wait(&bar->kv_full[s], (last_tile[s] / kStages) & 1, drain);
       }
@@ -217,187 +217,209 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (elect_one()) {
       const uint32_t idesc_qk = idesc_bf16(128, kNK, false, false);
       const uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
-      const uint32_t q_base = smem_u32(sQ);
-      int g = 0, piece = 0;
+      int g = 0, pc = 0;
       int row, k0, k1, nrow;
       bool first_row;
-      // P·V for tile t (A = P buffer, K-major; B = the stage's latent slabs, MN-major)
-      auto issue_pv = [&](int t, bool first, int pc) -> bool {
-        const int pb = t & 1, s = t % kStages;
-        if (!mbar_wait(&bar->p_full[pb], (t >> 1) & 1, guard)) return false;
+      // P·V for tile t: A = P in TMEM (aliasing the tile's score buffer), B = the stage's four
+      // latent slabs, MN-major (64 value columns per slab, keys along K).
+      auto issue_pv = [&](int t, bool first) -> bool {
+        const int sb = t % kNS, s = t % kStages;
+        if (!mbar_wait(&bar->p_full[sb], (t / kNS) & 1, guard)) return false;
         if (first && pc > 0 && !mbar_wait(&bar->o_empty, (pc - 1) & 1, guard)) return false;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sP + pb * kPBytes);
         const uint32_t b0 = smem_u32(sKV + s * kStageBytes);
 #pragma unroll
         for (int k = 0; k < kNK / 16; ++k) {
-          umma_bf16(tmem + kTmemO, smem_desc_sw128(a0 + k * 32, 16, 1024),
-                    smem_desc_sw128(b0 + k * 2048, kSlabKV, 1024), idesc_pv,
-                    (first && k == 0) ? 0u : 1u);
+          umma_bf16_tmem_a(tmem + kTmemO, tmem + kTmemS + sb * kNK + k * 8,
+                           smem_desc_sw128(b0 + k * 2048, kSlabKV, 1024), idesc_pv,
+                           (first && k == 0) ? 0u : 1u);
         }
         umma_commit(&bar->kv_empty[s]);
-        umma_commit(&bar->pv_done[pb]);
+        umma_commit(&bar->pv_done[sb]);
         return true;
       };
       bool ok = true;
       while (ok && it.get(row, k0, k1, nrow, first_row)) {
         const int ntiles = (k1 - k0 + kNK - 1) / kNK;
-        if (!mbar_wait(&bar->q_full, piece & 1, guard)) break;
+        if (!mbar_wait(&bar->q_full, pc & 1, guard)) break;
+        const int g0 = g;
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
-          const int s = g % kStages, sb = g & 1;
+          const int s = g % kStages, sb = g % kNS;
           if (!mbar_wait(&bar->kv_full[s], (g / kStages) & 1, guard)) { ok = false; break; }
-          if (g >= 2 && !mbar_wait(&bar->s_empty[sb], ((g >> 1) - 1) & 1, guard)) { ok = false; break; }
           tc_fence_after();
+          // scores: S[128 x 32] = Q_half (TMEM) x K_half^T (smem, K-major)
           const uint32_t kv0 = smem_u32(sKV + s * kStageBytes);
           for (int i = 0; i < nslabs; ++i) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              umma_bf16(tmem + kTmemS + sb * kNK,
-                        smem_desc_sw128(q_base + i * kSlabQ + kk * 32, 16, 1024),
-                        smem_desc_sw128(kv0 + i * kSlabKV + kk * 32, 16, 1024), idesc_qk,
-                        (i | kk) != 0);
+              umma_bf16_tmem_a(tmem + kTmemS + sb * kNK, tmem + kTmemQ + i * 32 + kk * 8,
+                               smem_desc_sw128(kv0 + i * kSlabKV + kk * 32, 16, 1024), idesc_qk,
+                               (i | kk) != 0);
             }
           }
           umma_commit(&bar->s_full[sb]);
           if (j == ntiles - 1) umma_commit(&bar->q_empty);
-          if (j > 0 && !issue_pv(g - 1, j - 1 == 0, piece)) { ok = false; break; }
+          if (j >= 2 && !issue_pv(g - 2, j - 2 == 0)) { ok = false; break; }
         }
         if (!ok) break;
-        if (!issue_pv(g - 1, ntiles == 1, piece)) break;
-        ++piece;
+        // the piece's last (up to two) P·V products
+        for (int t = (g - 2 > g0 ? g - 2 : g0); t < g && ok; ++t) ok = issue_pv(t, t == g0);
+        if (!ok) break;
+        ++pc;
         it.next();
       }
       umma_commit(&bar->drain);
     }
   } else {
-    // ---------------------------------------------------------------- softmax + epilogue
+    // ---------------------------------------------------------------- query load, softmax, epilogue
     const int quad = warp & 3;
     const int h = quad * 32 + static_cast<int>(lane_id());   // head row = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t x_remote = mapa_shared(smem_u32(sX), peer);
-    const uint32_t xfull_remote = mapa_shared(smem_u32(&bar->x_full), peer);
-    const uint32_t xempty_remote = mapa_shared(smem_u32(&bar->x_empty), peer);
+    const uint32_t x_local = smem_u32(sX);
+    const uint32_t x_remote = mapa_shared(x_local, peer);
+    const uint32_t xfull_remote[2] = {mapa_shared(smem_u32(&bar->x_full[0]), peer),
+                                      mapa_shared(smem_u32(&bar->x_full[1]), peer)};
+    const uint32_t xempty_remote[2] = {mapa_shared(smem_u32(&bar->x_empty[0]), peer),
+                                       mapa_shared(smem_u32(&bar->x_empty[1]), peer)};
     const int tid = static_cast<int>(threadIdx.x) - 64;     // 0..127
-    int g = 0, piece = 0;
+    const int nqw = rank == 0 ? 128 : 160;                  // query words (2 x bf16) per row
+    int g = 0, pc = 0;
     int row, k0, k1, nrow;
     bool first_row;
     bool ok = true;
-    while (ok && it.get(row, k0, k1, nrow, first_row)) {
-      const int ntiles = (k1 - k0 + kNK - 1) / kNK;
-      float m_run = -INFINITY, l_run = 0.f;
-      for (int j = 0; j < ntiles; ++j, ++g) {
-        const int sb = g & 1;
-        if (!mbar_wait(&bar->s_full[sb], (g >> 1) & 1, guard)) { ok = false; break; }
-        tc_fence_after();
-        float s[kNK];
-#pragma unroll
-        for (int c = 0; c < kNK / 16; ++c) {
-          float v[16];
-          tmem_ld16(tmem + lane_off + kTmemS + sb * kNK + c * 16, v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) s[c * 16 + i] = v[i];
-        }
-        tc_fence_before();
-        mbar_arrive(&bar->s_empty[sb]);
+    float m_run = -INFINITY, l_run = 0.f;
+    float prev[kNK];
 
-        // exchange the partial scores with the peer CTA
-        if (g >= 1 && !mbar_wait<true>(&bar->x_empty, (g - 1) & 1, guard)) { ok = false; break; }
+    // Finishes tile t (index jt within the piece): adds the peer's partial scores, runs the
+    // online softmax, writes P over the score buffer and frees the stage's invalid rows.
+    auto finish = [&](int t, int jt) -> bool {
+      const int xb = t & 1, sb = t % kNS;
+      if (tid == 0) mbar_arrive_expect_tx(&bar->x_full[xb], kXSlot);
+      if (!mbar_wait<true>(&bar->x_full[xb], (t >> 1) & 1, guard)) return false;
+      float s[kNK];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint32_t off = static_cast<uint32_t>(h * 256 + (((c + h) & 15) << 4));
-          st_cluster_v4(x_remote + off, s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
-        }
-        mbar_arrive_remote(xfull_remote);
-        if (!mbar_wait<true>(&bar->x_full, g & 1, guard)) { ok = false; break; }
+      for (int c = 0; c < kNK / 4; ++c) {
+        const float4 x = *reinterpret_cast<const float4*>(sX + xbuf_off(xb, h, c));
+        s[4 * c] = prev[4 * c] + x.x;
+        s[4 * c + 1] = prev[4 * c + 1] + x.y;
+        s[4 * c + 2] = prev[4 * c + 2] + x.z;
+        s[4 * c + 3] = prev[4 * c + 3] + x.w;
+      }
+      __syncwarp();
+      if (lane_id() == 0) mbar_arrive_remote_relaxed(xempty_remote[xb]);
+      const int key0 = k0 + jt * kNK;
+      const int nvalid = min(kNK, k1 - key0);
+      if (p.logits && rank == 0 && h < p.n_heads) {
+        float* lg = p.logits + (static_cast<size_t>(row) * p.n_heads + h) * p.max_seq_len + key0;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float4 x = *reinterpret_cast<const float4*>(
-              reinterpret_cast<const uint8_t*>(sX) + h * 256 + (((c + h) & 15) << 4));
-          s[4 * c] += x.x;
-          s[4 * c + 1] += x.y;
-          s[4 * c + 2] += x.z;
-          s[4 * c + 3] += x.w;
-        }
-        mbar_arrive_remote(xempty_remote);
-
-        // online softmax (log2 domain)
-        const int key0 = k0 + j * kNK;
-        const int nvalid = min(kNK, k1 - key0);
-        float mt = -INFINITY;
+        for (int i = 0; i < kNK; ++i)
+          if (i < nvalid) lg[i] = s[i] * p.scale;
+      }
+      float mt = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < kNK; ++i) {
-          const float x = i < nvalid ? s[i] * p.scale_log2 : -INFINITY;
-          s[i] = x;
-          mt = fmaxf(mt, x);
-        }
-        if (p.logits && rank == 0 && h < p.n_heads) {
-          float* lg = p.logits + (static_cast<size_t>(row) * p.n_heads + h) * p.max_seq_len + key0;
-          const float to_nat = p.scale / p.scale_log2;
-#pragma unroll
-          for (int i = 0; i < kNK; ++i)
-            if (i < nvalid) lg[i] = s[i] * to_nat;
-        }
-        const float m_new = fmaxf(m_run, mt);
-        if (m_new > m_run + kRescaleThreshold) {
-          if (j > 0) {
-            // O holds the earlier tiles: wait for their last P·V, then rescale the row in TMEM
-            if (!mbar_wait(&bar->pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, guard)) { ok = false; break; }
-            tc_fence_after();
-            const float f = exp2f(m_run - m_new);
-            l_run *= f;
+      for (int i = 0; i < kNK; ++i) {
+        s[i] = i < nvalid ? s[i] * p.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, s[i]);
+      }
+      // keep the pv_done phases of this buffer in step (P·V of tile t-3 has long finished)
+      if (t >= kNS && !mbar_wait(&bar->pv_done[sb], ((t / kNS) - 1) & 1, guard)) return false;
+      const float m_new = fmaxf(m_run, mt);
+      if (m_new > m_run + kRescaleThreshold) {
+        if (jt > 0) {
+          // O holds the earlier tiles of this piece: wait for their last P·V, rescale in TMEM
+          if (!mbar_wait(&bar->pv_done[(t - 1) % kNS], ((t - 1) / kNS) & 1, guard)) return false;
+          tc_fence_after();
+          const float f = fast_exp2(m_run - m_new);
+          l_run *= f;
 #pragma unroll 1
-            for (int c = 0; c < 256 / 16; ++c) {
-              float v[16];
-              tmem_ld16(tmem + lane_off + kTmemO + c * 16, v);
+          for (int c = 0; c < 256 / 16; ++c) {
+            float v[16];
+            tmem_ld16(tmem + lane_off + kTmemO + c * 16, v);
 #pragma unroll
-              for (int i = 0; i < 16; ++i) v[i] *= f;
-              tmem_st16(tmem + lane_off + kTmemO + c * 16, v);
-            }
+            for (int i = 0; i < 16; ++i) v[i] *= f;
+            tmem_st16(tmem + lane_off + kTmemO + c * 16, v);
           }
-          m_run = m_new;
         }
-        // P tile (bf16, K-major, 128-byte swizzle): row h, 16-byte chunk c at (c ^ (h & 7))
-        const int pb = g & 1;
-        if (g >= 2 && !mbar_wait(&bar->pv_done[pb], ((g >> 1) - 1) & 1, guard)) { ok = false; break; }
-        uint8_t* prow = sP + pb * kPBytes + h * 128;
-        float lsum = 0.f;
+        m_run = m_new;
+      }
+      uint32_t pk[kNK / 2];
+      float lsum = 0.f;
 #pragma unroll
-        for (int c = 0; c < kNK / 8; ++c) {
-          float e[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            e[i] = exp2f(s[c * 8 + i] - m_run);
-            lsum += e[i];
-          }
-          uint4 pk;
-          pk.x = pack_bf16x2(e[0], e[1]);
-          pk.y = pack_bf16x2(e[2], e[3]);
-          pk.z = pack_bf16x2(e[4], e[5]);
-          pk.w = pack_bf16x2(e[6], e[7]);
-          *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) = pk;
-        }
-        l_run += lsum;
-        if (nvalid < kNK) {
-          // keys past the row's end: zero their latent rows so garbage cannot reach P·V
-          uint8_t* st = sKV + (g % kStages) * kStageBytes;
-          const int nbytes_row = 128;
-          const int chunks = (kNK - nvalid) * (nbytes_row / 16) * 4;
-          for (int q = tid; q < chunks; q += 128) {
-            const int slab = q / ((kNK - nvalid) * 8);
-            const int rem = q - slab * ((kNK - nvalid) * 8);
-            const int r = nvalid + rem / 8;
-            const int ch = rem & 7;
-            *reinterpret_cast<uint4*>(st + slab * kSlabKV + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
-          }
+      for (int i = 0; i < kNK / 2; ++i) {
+        const float e0v = fast_exp2(s[2 * i] - m_run);
+        const float e1v = fast_exp2(s[2 * i + 1] - m_run);
+        lsum += e0v + e1v;
+        pk[i] = pack_bf16x2(e0v, e1v);
+      }
+      l_run += lsum;
+      tmem_st16_u32(tmem + lane_off + kTmemS + sb * kNK, pk);
+      if (nvalid < kNK) {
+        // keys past the piece's end: zero their latent rows so garbage cannot reach P·V
+        uint8_t* st = sKV + (t % kStages) * kStageBytes;
+        const int per_slab = (kNK - nvalid) * 8;
+        for (int q = tid; q < per_slab * 4; q += 128) {
+          const int slab = q / per_slab;
+          const int rem = q - slab * per_slab;
+          *reinterpret_cast<uint4*>(st + slab * kSlabKV + (nvalid + (rem >> 3)) * 128 +
+                                    ((rem & 7) << 4)) = make_uint4(0, 0, 0, 0);
         }
         fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(&bar->p_full[pb]);
+      }
+      tc_fence_before();
+      mbar_arrive(&bar->p_full[sb]);
+      return true;
+    };
+
+    while (ok && it.get(row, k0, k1, nrow, first_row)) {
+      const int ntiles = (k1 - k0 + kNK - 1) / kNK;
+      // this CTA's half of the absorbed query → TMEM (after the previous piece's last score MMA)
+      if (pc > 0 && !mbar_wait(&bar->q_empty, (pc - 1) & 1, guard)) break;
+      tc_fence_after();
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.qabs + (static_cast<size_t>(row) * kHPad + h) * kDk + col0);
+#pragma unroll 1
+        for (int c = 0; c < nqw / 16; ++c) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 v = __ldg(src + 4 * c + i);
+            w[4 * i] = v.x;
+            w[4 * i + 1] = v.y;
+            w[4 * i + 2] = v.z;
+            w[4 * i + 3] = v.w;
+          }
+          tmem_st16_u32(tmem + lane_off + kTmemQ + c * 16, w);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar->q_full);
+
+      m_run = -INFINITY;
+      l_run = 0.f;
+      for (int j = 0; j < ntiles; ++j, ++g) {
+        const int sb = g % kNS, xb = g & 1;
+        if (!mbar_wait(&bar->s_full[sb], (g / kNS) & 1, guard)) { ok = false; break; }
+        tc_fence_after();
+        float own[kNK];
+        tmem_ld32(tmem + lane_off + kTmemS + sb * kNK, own);
+        // send the partial scores of tile g to the peer
+        if (g >= 2 && !mbar_wait<true>(&bar->x_empty[xb], ((g >> 1) - 1) & 1, guard)) { ok = false; break; }
+#pragma unroll
+        for (int c = 0; c < kNK / 4; ++c)
+          st_async_v4(x_remote + xbuf_off(xb, h, c), own[4 * c], own[4 * c + 1], own[4 * c + 2],
+                      own[4 * c + 3], xfull_remote[xb]);
+        // finish the previous tile while this one's partner half is in flight
+        if (j > 0 && !finish(g - 1, j - 1)) { ok = false; break; }
+#pragma unroll
+        for (int i = 0; i < kNK; ++i) prev[i] = own[i];
       }
       if (!ok) break;
+      if (!finish(g - 1, ntiles - 1)) break;
+
       // ------------------------------------------------------------ epilogue of the piece
       const int glast = g - 1;
-      if (!mbar_wait(&bar->pv_done[glast & 1], (glast >> 1) & 1, guard)) break;
+      if (!mbar_wait(&bar->pv_done[glast % kNS], (glast / kNS) & 1, guard)) break;
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       const float lse = (m_run + log2f(l_run)) * 0.69314718055994531f;
@@ -405,21 +427,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (whole) {
         bf16* dst = p.o_lat + (static_cast<size_t>(row) * p.n_heads + h) * kC + col0;
 #pragma unroll 1
-        for (int c = 0; c < 256 / 16; ++c) {
-          float v[16];
-          tmem_ld16(tmem + lane_off + kTmemO + c * 16, v);
+        for (int c = 0; c < 256 / 32; ++c) {
+          float v[32];
+          tmem_ld32(tmem + lane_off + kTmemO + c * 32, v);
           if (h < p.n_heads) {
-            uint4 a, b;
-            a.x = pack_bf16x2(v[0] * inv_l, v[1] * inv_l);
-            a.y = pack_bf16x2(v[2] * inv_l, v[3] * inv_l);
-            a.z = pack_bf16x2(v[4] * inv_l, v[5] * inv_l);
-            a.w = pack_bf16x2(v[6] * inv_l, v[7] * inv_l);
-            b.x = pack_bf16x2(v[8] * inv_l, v[9] * inv_l);
-            b.y = pack_bf16x2(v[10] * inv_l, v[11] * inv_l);
-            b.z = pack_bf16x2(v[12] * inv_l, v[13] * inv_l);
-            b.w = pack_bf16x2(v[14] * inv_l, v[15] * inv_l);
-            reinterpret_cast<uint4*>(dst + c * 16)[0] = a;
-            reinterpret_cast<uint4*>(dst + c * 16)[1] = b;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 a;
+              a.x = pack_bf16x2(v[8 * q] * inv_l, v[8 * q + 1] * inv_l);
+              a.y = pack_bf16x2(v[8 * q + 2] * inv_l, v[8 * q + 3] * inv_l);
+              a.z = pack_bf16x2(v[8 * q + 4] * inv_l, v[8 * q + 5] * inv_l);
+              a.w = pack_bf16x2(v[8 * q + 6] * inv_l, v[8 * q + 7] * inv_l);
+              reinterpret_cast<uint4*>(dst + c * 32)[q] = a;
+            }
           }
         }
         if (rank == 0 && p.lse_out && h < p.n_heads)
@@ -428,19 +448,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int slot = first_row ? 0 : 1;
         float* dst = p.part_o + ((static_cast<size_t>(pair) * 2 + slot) * 128 + h) * kC + col0;
 #pragma unroll 1
-        for (int c = 0; c < 256 / 16; ++c) {
-          float v[16];
-          tmem_ld16(tmem + lane_off + kTmemO + c * 16, v);
+        for (int c = 0; c < 256 / 32; ++c) {
+          float v[32];
+          tmem_ld32(tmem + lane_off + kTmemO + c * 32, v);
 #pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + c * 16 + i) =
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + c * 32 + i) =
                 make_float4(v[i] * inv_l, v[i + 1] * inv_l, v[i + 2] * inv_l, v[i + 3] * inv_l);
         }
         if (rank == 0) p.part_lse[(static_cast<size_t>(pair) * 2 + slot) * 128 + h] = lse;
       }
       tc_fence_before();
       mbar_arrive(&bar->o_empty);
-      ++piece;
+      ++pc;
       it.next();
     }
   }
@@ -474,14 +494,15 @@ cudaError_t attention_prepare() {
                               kAttnSmem);
 }
 
-cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tpe,
-                             const AttnParams& p, int n_pairs, cudaStream_t s) {
-  latent_attention_kernel<<<dim3(2 * n_pairs), dim3(kThreads), kAttnSmem, s>>>(tq, tkv, tpe, p);
+cudaError_t launch_attention(const CUtensorMap& tkv, const CUtensorMap& tpe, const AttnParams& p,
+                             int n_pairs, cudaStream_t s) {
+  latent_attention_kernel<<<dim3(2 * n_pairs), dim3(kThreads), kAttnSmem, s>>>(tkv, tpe, p);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------------------------------
 // Combine: rows cut between pairs merge their normalised partials by log-sum-exp weights.
+// One warp per (row, head); lane l owns columns l, l+32, ..., l+480.
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ int pair_of_key(long long total, int pairs, long long e) {
   int q = static_cast<int>((e * pairs) / total);
@@ -491,46 +512,46 @@ __device__ __forceinline__ int pair_of_key(long long total, int pairs, long long
   return q;
 }
 
-__global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
+__global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   const int r = blockIdx.x;
+  const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (h >= p.n_heads) return;
   const long long total = p.row_prefix[p.rows];
   const int pairs = active_pairs(total, p.n_pairs, p.min_keys_per_pair);
   const long long R0 = p.row_prefix[r], R1 = p.row_prefix[r + 1];
   const int plo = pair_of_key(total, pairs, R0), phi = pair_of_key(total, pairs, R1 - 1);
   if (plo == phi) return;   // written by one pair
-  const int npart = phi - plo + 1;
-  for (int h = threadIdx.x >> 5; h < p.n_heads; h += 8) {
-    const int lane = threadIdx.x & 31;
-    float mx = -INFINITY;
-    for (int q = plo; q <= phi; ++q) {
-      const int slot = (q == plo && pair_begin(total, pairs, q) < R0) ? 1 : 0;
-      mx = fmaxf(mx, p.part_lse[(static_cast<size_t>(q) * 2 + slot) * 128 + h]);
-    }
-    float wsum = 0.f;
-    float acc[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-    for (int q = plo; q <= phi; ++q) {
-      const int slot = (q == plo && pair_begin(total, pairs, q) < R0) ? 1 : 0;
-      const size_t base = (static_cast<size_t>(q) * 2 + slot) * 128 + h;
-      const float w = exp2f((p.part_lse[base] - mx) * 1.4426950408889634f);
-      wsum += w;
-      const float* src = p.part_o + base * kC;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) acc[i] += w * src[lane + 32 * i];
-    }
-    (void)npart;
-    const float inv = 1.f / wsum;
-    bf16* dst = p.o_lat + (static_cast<size_t>(r) * p.n_heads + h) * kC;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) dst[lane + 32 * i] = __float2bfloat16_rn(acc[i] * inv);
-    if (lane == 0 && p.lse_out)
-      p.lse_out[static_cast<size_t>(r) * p.n_heads + h] = mx + logf(wsum);
+  float mx = -INFINITY;
+  for (int q = plo; q <= phi; ++q) {
+    const int slot = (q == plo && pair_begin(total, pairs, q) < R0) ? 1 : 0;
+    mx = fmaxf(mx, p.part_lse[(static_cast<size_t>(q) * 2 + slot) * 128 + h]);
   }
+  float wsum = 0.f;
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  for (int q = plo; q <= phi; ++q) {
+    const int slot = (q == plo && pair_begin(total, pairs, q) < R0) ? 1 : 0;
+    const size_t base = (static_cast<size_t>(q) * 2 + slot) * 128 + h;
+    const float w = exp2f((p.part_lse[base] - mx) * 1.4426950408889634f);
+    wsum += w;
+    const float* src = p.part_o + base * kC;
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __ldg(src + lane + 32 * i);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] = fmaf(w, v[i], acc[i]);
+  }
+  const float inv = 1.f / wsum;
+  bf16* dst = p.o_lat + (static_cast<size_t>(r) * p.n_heads + h) * kC;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) dst[lane + 32 * i] = __float2bfloat16_rn(acc[i] * inv);
+  if (lane == 0 && p.lse_out) p.lse_out[static_cast<size_t>(r) * p.n_heads + h] = mx + logf(wsum);
 }
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s) {
-  combine_kernel<<<p.rows, 256, 0, s>>>(p);
+  combine_kernel<<<dim3(p.rows, (p.n_heads + 3) / 4), 128, 0, s>>>(p);
   return cudaGetLastError();
 }
 
