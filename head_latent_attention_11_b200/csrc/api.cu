@@ -14,7 +14,7 @@
 
 #include <new>
 
-#include "../../include/mla.h"
+#include "mla.h"
 #include "internal.h"
 #include "tc100.cuh"
 

@@ -12,28 +12,32 @@
 //   * A cluster of TWO CTAs (one SM each) handles a row.  CTA 0 owns the latent columns
 //     [0, 256); CTA 1 owns [256, 512) and the 64 rotary columns.  Each CTA streams only its
 //     columns of every cache tile (the 576-wide cache row crosses HBM once), computes a partial
-//     score tile over them and sends it to the peer through distributed shared memory; both CTAs
-//     then hold identical full scores and run the identical online softmax.  Each CTA
-//     accumulates the value half it owns, O[128 x 256] fp32 in TMEM.
+//     score tile over them and hands it to the peer; both CTAs then hold identical full scores
+//     and run the identical online softmax.  Each CTA accumulates the value half it owns,
+//     O[128 x 256] fp32 in TMEM.
 //   * The CTA's half of the absorbed query lives in TMEM and is the A operand of the score MMA;
 //     the probabilities P (bf16) overwrite the score tile in TMEM and are the A operand of the
-//     P·V MMA.  Shared memory then holds only the cache ring (32-key tiles, 8 stages deep, TMA
-//     with 128-byte swizzle, evict-first) and the two exchange slots.
+//     P·V MMA.  Shared memory holds the cache ring (32-key tiles, 7 stages, TMA with 128-byte
+//     swizzle, evict-first) and the exchange buffers.
 //     TMEM columns: O [0,256) | query half [256,416) | three 32-column score/P buffers [416,512).
 //     With three buffers the score MMA of tile g only waits for P·V of tile g-3, so the tensor
 //     core runs two tiles ahead of the softmax.
-//   * The score exchange uses st.async: the partial scores land in the peer's shared memory and
-//     complete a transaction count on the peer's barrier, so the sender never stalls.  It is also
-//     software-pipelined: a thread sends tile g's partial scores, then finishes tile g-1 (whose
-//     partner half has arrived meanwhile).
+//   * Score exchange: partial tiles go through a local staging buffer to the bulk-copy engine
+//     (shared::cta → the peer's shared memory), which completes a transaction count on the
+//     peer's barrier.
+//   * Eight softmax warps in two groups of four that take alternate tiles (ping-pong); within a
+//     group one thread owns one head row.  Only the running-max decision is handed from tile to
+//     tile across the groups (per-row flag in shared memory); each group keeps its own partial
+//     row sum, so the softmax work of consecutive tiles overlaps.
+//   * Each warp stages its 32 rows of partial scores and ships them with its own 4 KB bulk copy.
 //   * The flattened key range of all rows is split evenly over the cluster pairs (split-K over
 //     keys, also across row boundaries); a row cut between pairs leaves normalised partials
 //     (O/l, lse) for the combine kernel, an uncut row is written as bf16 o_lat directly.
 //   * Online softmax in exp2 domain with lazy rescaling: the running max is only raised (and O
 //     in TMEM rescaled) when a tile's max exceeds it by more than 8 (factor 256), which keeps the
 //     rescale off the common path while the result stays exact.
-//   * Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-5 query loader,
-//     softmax and epilogue (thread = head row = TMEM lane).
+//   * Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-9 query loader,
+//     softmax and epilogue (thread pair = head row = TMEM lane).
 //   * Every wait is bounded (see tc100.cuh); a stuck pipeline records a status and ends.
 #include "internal.h"
 #include "tc100.cuh"
@@ -43,15 +47,17 @@ namespace mla {
 namespace {
 
 constexpr int kNK = kAttnKeysPerTile;      // keys per tile
-constexpr int kStages = 8;                 // cache tile ring depth
+constexpr int kStages = 7;                 // cache tile ring depth
 constexpr int kSlabKV = kNK * 128;         // 4 KB: 64 columns x 32 keys, bf16
 constexpr int kMaxSlabs = 5;               // rank 1: 4 latent slabs + 1 rotary slab
 constexpr int kStageBytes = kMaxSlabs * kSlabKV;
 constexpr int kXSlot = 128 * kNK * 4;      // 16 KB: one partial score tile, fp32
 
 constexpr int kOffKV = 0;
-constexpr int kOffX = kOffKV + kStages * kStageBytes;     // 160 KB
-constexpr int kOffBar = kOffX + 2 * kXSlot;               // 192 KB
+constexpr int kOffX = kOffKV + kStages * kStageBytes;     // receive slots (peer → this CTA)
+constexpr int kOffY = kOffX + 2 * kXSlot;                 // staging slots (this CTA → peer)
+constexpr int kOffRed = kOffY + 2 * kXSlot;               // row-max / row-sum exchange
+constexpr int kOffBar = kOffRed + 3 * 2 * 128 * 4;
 constexpr int kAttnSmem = kOffBar + 512 + 1024;
 
 constexpr int kTmemCols = 512;
@@ -60,20 +66,24 @@ constexpr uint32_t kTmemQ = 256;           // [256, 416): up to 320 bf16 K-colum
 constexpr uint32_t kTmemS = 416;           // three 32-column score / probability buffers
 constexpr int kNS = 3;
 
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
+constexpr int kThreads = 64 + kSoftmaxThreads;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_full, q_empty;
-  uint64_t s_full[kNS], p_full[kNS], pv_done[kNS];
+  uint64_t s_full[6], p_full[kNS], pv_done[6];
   uint64_t o_empty;
   uint64_t x_full[2], x_empty[2];
+  uint64_t sync_all;       // the 256 softmax threads
   uint64_t drain;
   uint32_t tmem_slot;
   int abort_flag;
 };
 static_assert(sizeof(Bars) <= 512, "barrier block");
+static_assert(kAttnSmem <= 232448, "shared memory budget");
 
 // Row containing flattened key e: largest r with prefix[r] <= e.
 __device__ __forceinline__ int row_of_key(const long long* prefix, int rows, long long e) {
@@ -126,6 +136,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sKV = smem + kOffKV;
   uint8_t* sX = smem + kOffX;
+  uint8_t* sY = smem + kOffY;
+  float* sRed = reinterpret_cast<float*>(smem + kOffRed);   // m_ref, seq, 2 x row sums
   Bars* bar = reinterpret_cast<Bars*>(smem + kOffBar);
 
   const uint32_t rank = cluster_ctarank();
@@ -147,18 +159,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&bar->kv_full[i], 1);
       mbar_init(&bar->kv_empty[i], 1);
     }
-    mbar_init(&bar->q_full, 128);
+    mbar_init(&bar->q_full, kSoftmaxThreads);
     mbar_init(&bar->q_empty, 1);
-    for (int i = 0; i < kNS; ++i) {
+    for (int i = 0; i < 6; ++i) {
       mbar_init(&bar->s_full[i], 1);
-      mbar_init(&bar->p_full[i], 128);
       mbar_init(&bar->pv_done[i], 1);
     }
+    for (int i = 0; i < kNS; ++i) mbar_init(&bar->p_full[i], 128);   // the tile's group
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar->x_full[i], 1);     // receiver's expect_tx arrival + the peer's bytes
-      mbar_init(&bar->x_empty[i], 4);    // one arrival per softmax warp of the peer
+      mbar_init(&bar->x_full[i], 1);     // receiver's expect_tx + the peer's four 4 KB copies
+      mbar_init(&bar->x_empty[i], 4);    // one arrival per warp of the peer's group
     }
-    mbar_init(&bar->o_empty, 128);
+    mbar_init(&bar->o_empty, kSoftmaxThreads);
+    mbar_init(&bar->sync_all, kSoftmaxThreads);
     mbar_init(&bar->drain, 1);
     bar->abort_flag = 0;
     fence_barrier_init();
@@ -235,7 +248,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                            (first && k == 0) ? 0u : 1u);
         }
         umma_commit(&bar->kv_empty[s]);
-        umma_commit(&bar->pv_done[sb]);
+        umma_commit(&bar->pv_done[t % 6]);
         return true;
       };
       bool ok = true;
@@ -257,7 +270,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                (i | kk) != 0);
             }
           }
-          umma_commit(&bar->s_full[sb]);
+          umma_commit(&bar->s_full[g % 6]);
           if (j == ntiles - 1) umma_commit(&bar->q_empty);
           if (j >= 2 && !issue_pv(g - 2, j - 2 == 0)) { ok = false; break; }
         }
@@ -272,164 +285,249 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- query load, softmax, epilogue
+    // Two groups of four warps take alternate tiles (group = global tile index & 1); within a
+    // group a thread owns one head row (TMEM lane) and all 32 keys of its tiles.  The running
+    // maximum of a row is handed from tile to tile across the groups through m_ref / seq in
+    // shared memory; each group keeps its own partial row sum relative to the last maximum it
+    // used, so the two groups' softmax work overlaps and only the max decision is sequential.
     const int quad = warp & 3;
-    const int h = quad * 32 + static_cast<int>(lane_id());   // head row = TMEM lane
+    const int grp = (warp - 2) >> 2;                         // 0: warps 2-5, 1: warps 6-9
+    const int lane = static_cast<int>(lane_id());
+    const int h = quad * 32 + lane;                          // head row = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t x_local = smem_u32(sX);
-    const uint32_t x_remote = mapa_shared(x_local, peer);
-    const uint32_t xfull_remote[2] = {mapa_shared(smem_u32(&bar->x_full[0]), peer),
-                                      mapa_shared(smem_u32(&bar->x_full[1]), peer)};
-    const uint32_t xempty_remote[2] = {mapa_shared(smem_u32(&bar->x_empty[0]), peer),
-                                       mapa_shared(smem_u32(&bar->x_empty[1]), peer)};
-    const int tid = static_cast<int>(threadIdx.x) - 64;     // 0..127
-    const int nqw = rank == 0 ? 128 : 160;                  // query words (2 x bf16) per row
+    const int tid = static_cast<int>(threadIdx.x) - 64;      // 0..255
+    const int gtid = tid & 127;                              // thread index within the group
+    volatile float* m_ref = reinterpret_cast<volatile float*>(sRed);            // [128]
+    volatile int* seq = reinterpret_cast<volatile int*>(sRed + 128);            // [128]
+    float* lsum_x = sRed + 256;                                                  // [2][128]
+    const uint32_t y_warp = smem_u32(sY) + grp * kXSlot + quad * 4096;         // this warp's rows
+    const uint32_t x_warp_remote = mapa_shared(smem_u32(sX), peer) + grp * kXSlot + quad * 4096;
+    const uint32_t xfull_remote = mapa_shared(smem_u32(&bar->x_full[grp]), peer);
+    const uint32_t xempty_remote = mapa_shared(smem_u32(&bar->x_empty[grp]), peer);
+    const int nqw = rank == 0 ? 128 : 160;                   // query words (2 x bf16) per row
     int g = 0, pc = 0;
     int row, k0, k1, nrow;
     bool first_row;
     bool ok = true;
-    float m_run = -INFINITY, l_run = 0.f;
-    float prev[kNK];
-
-    // Finishes tile t (index jt within the piece): adds the peer's partial scores, runs the
-    // online softmax, writes P over the score buffer and frees the stage's invalid rows.
-    auto finish = [&](int t, int jt) -> bool {
-      const int xb = t & 1, sb = t % kNS;
-      if (tid == 0) mbar_arrive_expect_tx(&bar->x_full[xb], kXSlot);
-      if (!mbar_wait<true>(&bar->x_full[xb], (t >> 1) & 1, guard)) return false;
-      float s[kNK];
-#pragma unroll
-      for (int c = 0; c < kNK / 4; ++c) {
-        const float4 x = *reinterpret_cast<const float4*>(sX + xbuf_off(xb, h, c));
-        s[4 * c] = prev[4 * c] + x.x;
-        s[4 * c + 1] = prev[4 * c + 1] + x.y;
-        s[4 * c + 2] = prev[4 * c + 2] + x.z;
-        s[4 * c + 3] = prev[4 * c + 3] + x.w;
-      }
-      __syncwarp();
-      if (lane_id() == 0) mbar_arrive_remote_relaxed(xempty_remote[xb]);
-      const int key0 = k0 + jt * kNK;
-      const int nvalid = min(kNK, k1 - key0);
-      if (p.logits && rank == 0 && h < p.n_heads) {
-        float* lg = p.logits + (static_cast<size_t>(row) * p.n_heads + h) * p.max_seq_len + key0;
-#pragma unroll
-        for (int i = 0; i < kNK; ++i)
-          if (i < nvalid) lg[i] = s[i] * p.scale;
-      }
-      float mt = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < kNK; ++i) {
-        s[i] = i < nvalid ? s[i] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, s[i]);
-      }
-      // keep the pv_done phases of this buffer in step (P·V of tile t-3 has long finished)
-      if (t >= kNS && !mbar_wait(&bar->pv_done[sb], ((t / kNS) - 1) & 1, guard)) return false;
-      const float m_new = fmaxf(m_run, mt);
-      if (m_new > m_run + kRescaleThreshold) {
-        if (jt > 0) {
-          // O holds the earlier tiles of this piece: wait for their last P·V, rescale in TMEM
-          if (!mbar_wait(&bar->pv_done[(t - 1) % kNS], ((t - 1) / kNS) & 1, guard)) return false;
-          tc_fence_after();
-          const float f = fast_exp2(m_run - m_new);
-          l_run *= f;
-#pragma unroll 1
-          for (int c = 0; c < 256 / 16; ++c) {
-            float v[16];
-            tmem_ld16(tmem + lane_off + kTmemO + c * 16, v);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] *= f;
-            tmem_st16(tmem + lane_off + kTmemO + c * 16, v);
-          }
-        }
-        m_run = m_new;
-      }
-      uint32_t pk[kNK / 2];
-      float lsum = 0.f;
-#pragma unroll
-      for (int i = 0; i < kNK / 2; ++i) {
-        const float e0v = fast_exp2(s[2 * i] - m_run);
-        const float e1v = fast_exp2(s[2 * i + 1] - m_run);
-        lsum += e0v + e1v;
-        pk[i] = pack_bf16x2(e0v, e1v);
-      }
-      l_run += lsum;
-      tmem_st16_u32(tmem + lane_off + kTmemS + sb * kNK, pk);
-      if (nvalid < kNK) {
-        // keys past the piece's end: zero their latent rows so garbage cannot reach P·V
-        uint8_t* st = sKV + (t % kStages) * kStageBytes;
-        const int per_slab = (kNK - nvalid) * 8;
-        for (int q = tid; q < per_slab * 4; q += 128) {
-          const int slab = q / per_slab;
-          const int rem = q - slab * per_slab;
-          *reinterpret_cast<uint4*>(st + slab * kSlabKV + (nvalid + (rem >> 3)) * 128 +
-                                    ((rem & 7) << 4)) = make_uint4(0, 0, 0, 0);
-        }
-        fence_async_smem();
-      }
-      tc_fence_before();
-      mbar_arrive(&bar->p_full[sb]);
-      return true;
+    uint32_t ph_all = 0;
+    auto sync_all = [&]() -> bool {
+      mbar_arrive(&bar->sync_all);
+      return warp_wait(&bar->sync_all, (ph_all++) & 1, guard);
     };
+    if (tid < 128) seq[tid] = -1;
+    if (!sync_all()) ok = false;
 
     while (ok && it.get(row, k0, k1, nrow, first_row)) {
       const int ntiles = (k1 - k0 + kNK - 1) / kNK;
-      // this CTA's half of the absorbed query → TMEM (after the previous piece's last score MMA)
-      if (pc > 0 && !mbar_wait(&bar->q_empty, (pc - 1) & 1, guard)) break;
-      tc_fence_after();
+      const int g0 = g;
+      // this CTA's half of the absorbed query → TMEM (after the previous piece's last score
+      // MMA); the two threads of a row (one per group) split its words, all loads in flight
       {
+        const int nw = nqw / 2;                              // 64 or 80 words per thread
         const uint4* src = reinterpret_cast<const uint4*>(
-            p.qabs + (static_cast<size_t>(row) * kHPad + h) * kDk + col0);
-#pragma unroll 1
-        for (int c = 0; c < nqw / 16; ++c) {
-          uint32_t w[16];
+            p.qabs + (static_cast<size_t>(row) * kHPad + h) * kDk + col0) + grp * (nw / 4);
+        uint32_t w[80];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 v = __ldg(src + 4 * c + i);
+        for (int i = 0; i < 20; ++i) {
+          if (i < nw / 4) {
+            const uint4 v = __ldg(src + i);
             w[4 * i] = v.x;
             w[4 * i + 1] = v.y;
             w[4 * i + 2] = v.z;
             w[4 * i + 3] = v.w;
           }
-          tmem_st16_u32(tmem + lane_off + kTmemQ + c * 16, w);
+        }
+        if (pc > 0 && !warp_wait(&bar->q_empty, (pc - 1) & 1, guard)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 5; ++c) {
+          if (c < nw / 16) {
+            uint32_t ww[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ww[i] = w[16 * c + i];
+            tmem_st16_u32(tmem + lane_off + kTmemQ + grp * nw + c * 16, ww);
+          }
         }
       }
       tc_fence_before();
       mbar_arrive(&bar->q_full);
 
-      m_run = -INFINITY;
-      l_run = 0.f;
-      for (int j = 0; j < ntiles; ++j, ++g) {
-        const int sb = g % kNS, xb = g & 1;
-        if (!mbar_wait(&bar->s_full[sb], (g / kNS) & 1, guard)) { ok = false; break; }
+      float l_g = 0.f;              // this group's partial row sum ...
+      float m_used = -INFINITY;     // ... relative to this maximum
+      int j = ((g0 & 1) == grp) ? 0 : 1;
+      for (; j < ntiles; j += 2) {
+        const int t = g0 + j;
+        const int k = t >> 1;       // per-group tile counter (exchange slot phases)
+        // scores of this CTA's columns
+        if (!warp_wait(&bar->s_full[t % 6], (t / 6) & 1, guard)) { ok = false; break; }
         tc_fence_after();
-        float own[kNK];
-        tmem_ld32(tmem + lane_off + kTmemS + sb * kNK, own);
-        // send the partial scores of tile g to the peer
-        if (g >= 2 && !mbar_wait<true>(&bar->x_empty[xb], ((g >> 1) - 1) & 1, guard)) { ok = false; break; }
+        float s[kNK];
+        tmem_ld32(tmem + lane_off + kTmemS + (t % kNS) * kNK, s);
+        // hand this warp's 32 rows to the peer: stage locally, one bulk copy per warp
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
 #pragma unroll
         for (int c = 0; c < kNK / 4; ++c)
-          st_async_v4(x_remote + xbuf_off(xb, h, c), own[4 * c], own[4 * c + 1], own[4 * c + 2],
-                      own[4 * c + 3], xfull_remote[xb]);
-        // finish the previous tile while this one's partner half is in flight
-        if (j > 0 && !finish(g - 1, j - 1)) { ok = false; break; }
+          *reinterpret_cast<float4*>(sY + grp * kXSlot + xbuf_off(0, h, c)) =
+              make_float4(s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (k >= 1 && !mbar_wait<true>(&bar->x_empty[grp], (k - 1) & 1, guard)) ok = false;
+          if (ok) {
+            bulk_copy_to_peer(x_warp_remote, y_warp, 4096, xfull_remote);
+            bulk_commit();
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        // the peer's half of the same tile
+        if (gtid == 0) mbar_arrive_expect_tx(&bar->x_full[grp], kXSlot);
+        if (!warp_wait<true>(&bar->x_full[grp], k & 1, guard)) { ok = false; break; }
 #pragma unroll
-        for (int i = 0; i < kNK; ++i) prev[i] = own[i];
+        for (int c = 0; c < kNK / 4; ++c) {
+          const float4 x =
+              *reinterpret_cast<const float4*>(sX + grp * kXSlot + xbuf_off(0, h, c));
+          s[4 * c] += x.x;
+          s[4 * c + 1] += x.y;
+          s[4 * c + 2] += x.z;
+          s[4 * c + 3] += x.w;
+        }
+        // every lane has consumed its loads from the slot before lane 0 lets the peer refill it
+        consume32(s);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote_relaxed(xempty_remote);
+        const int key0 = k0 + j * kNK;
+        const int nvalid = min(kNK, k1 - key0);
+        if (p.logits && rank == 0 && h < p.n_heads) {
+          float* lg =
+              p.logits + (static_cast<size_t>(row) * p.n_heads + h) * p.max_seq_len + key0;
+#pragma unroll
+          for (int i = 0; i < kNK; ++i)
+            if (i < nvalid) lg[i] = s[i] * p.scale;
+        }
+        float mx[8];
+#pragma unroll
+        for (int i = 0; i < kNK; ++i) s[i] = i < nvalid ? s[i] * p.scale_log2 : -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(fmaxf(s[i], s[i + 8]), fmaxf(s[i + 16], s[i + 24]));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
+        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        // running-max decision for tile t (after the other group decided tile t-1)
+        float m_prev = -INFINITY;
+        if (j > 0) {
+          bool seen = true;
+          if (seq[h] != t - 1) {
+            const unsigned long long t0 = globaltimer_ns();
+            uint32_t n = 0;
+            while (seq[h] != t - 1) {
+              if ((++n & 63u) == 0 &&
+                  (guard.aborted() || globaltimer_ns() - t0 > kWaitLimitNs)) {
+                if (!guard.aborted()) guard.fail(kDevTimeout);
+                seen = false;
+                break;
+              }
+            }
+          }
+          if (!__all_sync(0xffffffffu, seen)) { ok = false; break; }
+          __threadfence_block();
+          m_prev = m_ref[h];
+        }
+        float m_dec = m_prev;
+        const float m_new = fmaxf(m_prev, mt);
+        const bool raise = m_new > m_prev + kRescaleThreshold;
+        // O holds tiles up to t-1: if any row of the warp raises its maximum, the warp waits for
+        // their last P·V and rescales (factor 1 for the other rows) — warp-uniform TMEM access
+        if (j > 0 && __any_sync(0xffffffffu, raise)) {
+          if (!warp_wait(&bar->pv_done[(t - 1) % 6], ((t - 1) / 6) & 1, guard)) { ok = false; break; }
+          tc_fence_after();
+          const float f = raise ? fast_exp2(m_prev - m_new) : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < 256 / 16; ++c) {
+            float v[16];
+            const uint32_t a = tmem + lane_off + kTmemO + c * 16;
+            tmem_ld16(a, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] *= f;
+            tmem_st16(a, v);
+          }
+          tc_fence_before();
+        }
+        if (raise) m_dec = m_new;
+        m_ref[h] = m_dec;
+        __threadfence_block();
+        seq[h] = t;
+        if (m_used != m_dec) {
+          if (m_used != -INFINITY) l_g *= fast_exp2(m_used - m_dec);
+          m_used = m_dec;
+        }
+        // probabilities → TMEM (over the score buffer), row sum
+        uint32_t pk[kNK / 2];
+        float e[kNK];
+#pragma unroll
+        for (int i = 0; i < kNK; ++i) e[i] = fast_exp2(s[i] - m_dec);
+#pragma unroll
+        for (int i = 0; i < kNK / 2; ++i) pk[i] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) e[i] += e[i + 16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) e[i] += e[i + 8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) e[i] += e[i + 4];
+        l_g += (e[0] + e[2]) + (e[1] + e[3]);
+        tmem_st16_u32(tmem + lane_off + kTmemS + (t % kNS) * kNK, pk);
+        if (nvalid < kNK) {
+          // keys past the piece's end: zero their latent rows so garbage cannot reach P·V
+          uint8_t* st = sKV + (t % kStages) * kStageBytes;
+          const int per_slab = (kNK - nvalid) * 8;
+          for (int q = gtid; q < per_slab * 4; q += 128) {
+            const int slab = q / per_slab;
+            const int rem = q - slab * per_slab;
+            *reinterpret_cast<uint4*>(st + slab * kSlabKV + (nvalid + (rem >> 3)) * 128 +
+                                      ((rem & 7) << 4)) = make_uint4(0, 0, 0, 0);
+          }
+          fence_async_smem();
+        }
+        tc_fence_before();
+        mbar_arrive(&bar->p_full[t % kNS]);
       }
       if (!ok) break;
-      if (!finish(g - 1, ntiles - 1)) break;
+      g = g0 + ntiles;
 
       // ------------------------------------------------------------ epilogue of the piece
       const int glast = g - 1;
-      if (!mbar_wait(&bar->pv_done[glast % kNS], (glast / kNS) & 1, guard)) break;
+      // final maximum of the row (decided at the last tile), both groups' sums relative to it
+      {
+        bool seen = true;
+        const unsigned long long t0 = globaltimer_ns();
+        uint32_t n = 0;
+        while (seq[h] != glast) {
+          if ((++n & 63u) == 0 && (guard.aborted() || globaltimer_ns() - t0 > kWaitLimitNs)) {
+            if (!guard.aborted()) guard.fail(kDevTimeout);
+            seen = false;
+            break;
+          }
+        }
+        if (!__all_sync(0xffffffffu, seen)) break;
+      }
+      __threadfence_block();
+      const float m_fin = m_ref[h];
+      lsum_x[grp * 128 + h] = (m_used == -INFINITY) ? 0.f : l_g * fast_exp2(m_used - m_fin);
+      if (!sync_all()) break;
+      const float l_tot = lsum_x[h] + lsum_x[128 + h];
+      if (!warp_wait(&bar->pv_done[glast % 6], (glast / 6) & 1, guard)) break;
       tc_fence_after();
-      const float inv_l = 1.f / l_run;
-      const float lse = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      const float inv_l = 1.f / l_tot;
+      const float lse = (m_fin + log2f(l_tot)) * 0.69314718055994531f;
       const bool whole = (k0 == 0 && k1 == nrow);
+      const int ocol = col0 + grp * 128;
       if (whole) {
-        bf16* dst = p.o_lat + (static_cast<size_t>(row) * p.n_heads + h) * kC + col0;
+        bf16* dst = p.o_lat + (static_cast<size_t>(row) * p.n_heads + h) * kC + ocol;
 #pragma unroll 1
-        for (int c = 0; c < 256 / 32; ++c) {
+        for (int c = 0; c < 128 / 32; ++c) {
           float v[32];
-          tmem_ld32(tmem + lane_off + kTmemO + c * 32, v);
+          tmem_ld32(tmem + lane_off + kTmemO + grp * 128 + c * 32, v);
           if (h < p.n_heads) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -442,27 +540,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (rank == 0 && p.lse_out && h < p.n_heads)
+        if (rank == 0 && grp == 0 && p.lse_out && h < p.n_heads)
           p.lse_out[static_cast<size_t>(row) * p.n_heads + h] = lse;
       } else {
         const int slot = first_row ? 0 : 1;
-        float* dst = p.part_o + ((static_cast<size_t>(pair) * 2 + slot) * 128 + h) * kC + col0;
+        float* dst = p.part_o + ((static_cast<size_t>(pair) * 2 + slot) * 128 + h) * kC + ocol;
 #pragma unroll 1
-        for (int c = 0; c < 256 / 32; ++c) {
+        for (int c = 0; c < 128 / 32; ++c) {
           float v[32];
-          tmem_ld32(tmem + lane_off + kTmemO + c * 32, v);
+          tmem_ld32(tmem + lane_off + kTmemO + grp * 128 + c * 32, v);
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4*>(dst + c * 32 + i) =
                 make_float4(v[i] * inv_l, v[i + 1] * inv_l, v[i + 2] * inv_l, v[i + 3] * inv_l);
         }
-        if (rank == 0) p.part_lse[(static_cast<size_t>(pair) * 2 + slot) * 128 + h] = lse;
+        if (rank == 0 && grp == 0)
+          p.part_lse[(static_cast<size_t>(pair) * 2 + slot) * 128 + h] = lse;
       }
       tc_fence_before();
       mbar_arrive(&bar->o_empty);
       ++pc;
       it.next();
     }
+    if (lane == 0) bulk_wait_all();   // every copy this warp sent has landed in the peer
   }
 
   // ------------------------------------------------------------------ teardown

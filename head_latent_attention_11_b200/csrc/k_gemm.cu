@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int quad = warp & 3;
     const int row = quad * 32 + static_cast<int>(lane_id());
     const int m = m0 + row;
-    const bool ok = mbar_wait(dfull, 0, guard);
+    const bool ok = warp_wait(dfull, 0, guard);   // converged warp for tcgen05.ld
     tc_fence_after();
     if (ok) {
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16);

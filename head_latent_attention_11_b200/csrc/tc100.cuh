@@ -130,6 +130,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Whole-warp wait: every lane polls, then the lanes vote, so the warp leaves converged and
+// agrees on the outcome (tcgen05.ld/st that follow are .sync.aligned and need the whole warp).
+template <bool kClusterAcquire = false>
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Guard& g) {
+  const bool ok = mbar_wait<kClusterAcquire>(bar, parity, g);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ------------------------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor) — tile loads into this CTA's shared memory, no multicast
 // ------------------------------------------------------------------------------------------
@@ -175,10 +183,13 @@ __device__ __forceinline__ void fence_async_smem() {
 }
 
 // ------------------------------------------------------------------------------------------
-// Tensor memory
+// Tensor memory.  tcgen05.alloc/dealloc/ld/st are .sync.aligned: every lane of the warp must
+// execute them together, so each helper first reconverges the warp; callers keep them out of
+// lane-dependent branches.
 // ------------------------------------------------------------------------------------------
 // Executed by one full warp; writes the TMEM base address into *dst_smem.
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  __syncwarp();   // .sync.aligned: the whole warp, converged
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(dst_smem)),
                "r"(ncols)
@@ -187,6 +198,7 @@ __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
 }
 
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  __syncwarp();   // .sync.aligned: the whole warp, converged
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
@@ -203,6 +215,7 @@ __device__ __forceinline__ void tc_fence_after() {
 // registers before the data has arrived.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
+  __syncwarp();   // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
       "%14,%15}, [%16];\n\t"
@@ -218,6 +231,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 
 // Store 16 columns and wait for the store to land.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  __syncwarp();   // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
       "%13,%14,%15,%16};\n\t"
@@ -234,6 +248,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
 
 // Raw 32-bit words to TMEM (16 columns) and wait for the store.
 __device__ __forceinline__ void tmem_st16_u32(uint32_t taddr, const uint32_t (&r)[16]) {
+  __syncwarp();   // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
       "%13,%14,%15,%16};\n\t"
@@ -243,9 +258,20 @@ __device__ __forceinline__ void tmem_st16_u32(uint32_t taddr, const uint32_t (&r
       : "memory");
 }
 
+// 8 raw 32-bit words to TMEM and wait for the store.
+__device__ __forceinline__ void tmem_st8_u32(uint32_t taddr, const uint32_t (&r)[8]) {
+  __syncwarp();   // .sync.aligned: the whole warp, converged
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 // 32 lanes x 32 bit, 32 consecutive columns per thread, load + wait fused.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
+  __syncwarp();   // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
       "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
@@ -363,13 +389,52 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, float a, float
 }
 
 // Arrive on a barrier of another CTA of the cluster without ordering earlier memory operations.
+// Callers that use it to release a buffer first consume every value they loaded from it (see
+// consume32), so the loads have completed before this instruction can issue.
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar_addr) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
                    remote_bar_addr)
                : "memory");
 }
 
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory to another CTA's shared
+// memory in the cluster; on arrival it performs complete_tx(bytes) on the remote barrier.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t remote_dst, uint32_t local_src,
+                                                  uint32_t bytes, uint32_t remote_bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(remote_dst), "r"(local_src), "r"(bytes), "r"(remote_bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every committed bulk copy of this thread has finished reading its source.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Wait until every committed bulk copy of this thread has completed (destination written).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Named barrier over `nthreads` threads (whole warps).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Makes the 32 values "used" at this point in program order: the instructions producing them
+// (and the loads they depend on) are scheduled before anything that follows.
+__device__ __forceinline__ void consume32(const float (&v)[32]) {
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) acc += v[i] * 0.f;
+  asm volatile("" ::"f"(acc) : "memory");
+}
+
 __device__ __forceinline__ void cluster_sync_all() {
+  __syncwarp();   // .aligned: converged warps
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
 }

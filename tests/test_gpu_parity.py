@@ -134,6 +134,31 @@ def test_decode_edges(H, B, L):
     _decode_case(w, seed=H + B + L, tail="nan")
 
 
+def test_decode_repeat_is_bitwise_stable():
+    """Rows cut across SM pairs, debug logits on (which skews the two CTAs of a pair): repeated
+    calls must give bit-identical results within the bound (guards the score exchange)."""
+    from mla_synth import MLADims
+    w = workload("tiny_decode", dims=MLADims(128), batch=7, cache_len=300)
+    inp = make_inputs(w, seed=435, tail="nan")
+    dev = to_device(inp)
+    rt = _runtime(dev, w, w.batch, inp["max_t"])
+    ref = oracle_decode(inp, w)
+    logits = torch.full((w.batch, 128, inp["max_t"]), float("nan"), device="cuda")
+    first = None
+    for _ in range(12):
+        out = rt.decode(dev["q_latent"].reshape(w.batch, -1), dev["start_pos"], dev["cache"],
+                        logits=logits)
+        torch.cuda.synchronize()
+        got = bf16_to_np(out)
+        if first is None:
+            first = got
+            assert_close_bf16(f64(out), ref["out"], "repeat out")
+        else:
+            assert np.array_equal(got, first), "results differ between identical calls"
+    assert rt.sync_status() == 0
+    rt.close()
+
+
 def test_decode_ragged_small():
     from mla_synth import MLADims
     w = workload("ragged_decode", dims=MLADims(128), batch=6, ragged=(1, 3000))
