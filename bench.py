@@ -70,6 +70,26 @@ def measured_peaks() -> dict:
 
 
 # ------------------------------------------------------------------------------------------
+# Multi-rank aggregation (replicas: every rank runs its own batch, no data exchange)
+# ------------------------------------------------------------------------------------------
+def max_over_ranks(values, device="cpu"):
+    """Element-wise max of per-rank float values over the default process group (a no-op when
+    torch.distributed is not initialised).  Only timings cross ranks; the data path has no
+    collective."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def aggregate_throughput(units_per_rank: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: all ranks' units over the slowest rank's timed region."""
+    return world * units_per_rank * steps / (max_ms / 1e3)
+
+
+# ------------------------------------------------------------------------------------------
 # Clock sampling during the timed region
 # ------------------------------------------------------------------------------------------
 class ClockSampler:
@@ -236,10 +256,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     d2h = h_out.numel() * 2
 
     # ---- max over ranks
-    t = torch.tensor([total_ms, float(np.sum(e2e_ms))], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_total = float(t[0]), float(t[1])
+    total_ms, e2e_total = max_over_ranks([total_ms, float(np.sum(e2e_ms))], device=dev)
     rt.close()
     if rank != 0:
         return None
@@ -248,9 +265,9 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     ms_per_step = total_ms / args.steps
     units = B * T
     if w.mode == "decode":
-        value = world * units * args.steps / (total_ms / 1e3)
+        value = aggregate_throughput(units, args.steps, world, total_ms)
         unit = "queries/s"
-        e2e_value = world * units * args.steps / (e2e_total / 1e3)
+        e2e_value = aggregate_throughput(units, args.steps, world, e2e_total)
     else:
         value = world * work["flops"] * args.steps / (total_ms / 1e3) / 1e12
         unit = "TFLOP/s"
