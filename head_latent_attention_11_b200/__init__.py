@@ -18,7 +18,7 @@ __all__ = [
     "MLAError", "MLAConfig", "load", "lib_path", "mla_status_string", "mla_workspace_size",
     "mla_init", "mla_destroy", "mla_rmsnorm", "mla_decode", "mla_prefill_chunk", "mla_sync_status",
     "mla_enable_stage_timing", "mla_stage_times", "mla_debug_copy", "mla_last_launch_count",
-    "EXPORTED_SYMBOLS", "STATUS",
+    "EXPORTED_SYMBOLS", "STATUS", "mla_latent_attention_noalloc",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,6 +33,7 @@ EXPORTED_SYMBOLS = (
     "mla_status_string", "mla_workspace_size", "mla_init", "mla_destroy", "mla_rmsnorm",
     "mla_decode", "mla_prefill_chunk", "mla_sync_status", "mla_enable_stage_timing",
     "mla_stage_times", "mla_debug_copy", "mla_last_launch_count",
+    "mla_latent_attention_noalloc",
 )
 
 
@@ -96,6 +97,8 @@ def load() -> ctypes.CDLL:
                                            ctypes.POINTER(I32)]),
         "mla_debug_copy": (ctypes.c_int, [P, I32, P, SZ, P]),
         "mla_last_launch_count": (I32, [P]),
+        "mla_latent_attention_noalloc": (ctypes.c_int, [P, P, I32, I32, F, P, I64, I64, P, I64,
+                                                        I64, I32, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -198,3 +201,15 @@ def mla_debug_copy(ctx, which: int, dst, nbytes: int, stream=None) -> None:
 
 def mla_last_launch_count(ctx) -> int:
     return int(load().mla_last_launch_count(ctx))
+
+
+def mla_latent_attention_noalloc(q_abs, start_pos, rows: int, n_heads: int, softmax_scale: float,
+                                 kv_cache, kv_stride_b: int, kv_stride_t: int, pe_cache,
+                                 pe_stride_b: int, pe_stride_t: int, max_seq_len: int, o_lat,
+                                 lse=None, status=None, stream=None) -> None:
+    """Attention over the cache for given absorbed queries using no memory beyond the arguments
+    and the library's fixed scratch array (see include/mla.h for limits and set-up)."""
+    _check("mla_latent_attention_noalloc", load().mla_latent_attention_noalloc(
+        _ptr(q_abs), _ptr(start_pos), rows, n_heads, softmax_scale, _ptr(kv_cache), kv_stride_b,
+        kv_stride_t, _ptr(pe_cache), pe_stride_b, pe_stride_t, max_seq_len, _ptr(o_lat),
+        _ptr(lse), _ptr(status), _stream(stream)))

@@ -102,6 +102,7 @@ struct CombineParams {
 
 // Launchers (defined next to their kernels).
 cudaError_t launch_rmsnorm(const RmsParams& p, cudaStream_t s);
+cudaError_t launch_key_prefix(const RmsParams& p, cudaStream_t s);   // row_prefix only
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                         int batches, cudaStream_t s);
 cudaError_t launch_attention(const CUtensorMap& tkv, const CUtensorMap& tpe, const AttnParams& p,

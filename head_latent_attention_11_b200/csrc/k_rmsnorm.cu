@@ -140,4 +140,13 @@ cudaError_t launch_rmsnorm(const RmsParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Cumulative key counts of decode rows only (one block); used by the no-allocation attention
+// entry point, which has no RMSNorm launch to carry it.
+__global__ void __launch_bounds__(128) key_prefix_kernel(const RmsParams p) { key_prefix_block(p); }
+
+cudaError_t launch_key_prefix(const RmsParams& p, cudaStream_t s) {
+  key_prefix_kernel<<<1, 128, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
 }  // namespace mla

@@ -1,0 +1,164 @@
+// noalloc.cu — latent attention entry point that allocates no memory.
+//
+// Some callers cannot allocate device memory at the point where they run attention: code that
+// runs inside a pre-reserved memory pool it must not grow, plug-ins handed a fixed device budget
+// by their host, or a process whose allocator is owned by another framework.  This entry point
+// serves them: the caller passes its inputs and outputs, and the only other device memory used
+// is the fixed scratch array below, part of the library's image on every device that loads it.
+//
+// The scratch holds the per-row key prefix, the split-K partial outputs of at most
+// kNoAllocPairs SM pairs and a status word.  Limits: rows <= kNoAllocMaxRows; the attention
+// splits over at most kNoAllocPairs pairs (fewer SMs than the context path on large GPUs).
+//
+// Set-up: the first call on a device (with that device current) resolves the array's device
+// address with cudaGetSymbolAddress and sets the attention kernel's shared-memory attribute;
+// make that first call before capturing the stream into a CUDA graph.  Every call shares the
+// same array, so calls that may overlap on the GPU (different streams, different threads)
+// race on it and must be serialised by the caller.
+#include <mutex>
+
+#include "mla.h"
+#include "internal.h"
+#include "tc100.cuh"
+
+namespace mla {
+namespace {
+
+constexpr int kNoAllocMaxRows = 4096;
+constexpr int kNoAllocPairs = 16;
+constexpr size_t kOffStatus = 0;
+constexpr size_t kOffPrefix = 256;
+constexpr size_t kOffPartO = kOffPrefix + ((static_cast<size_t>(kNoAllocMaxRows) + 1) * 8 + 255) / 256 * 256;
+constexpr size_t kOffPartLse = kOffPartO + static_cast<size_t>(kNoAllocPairs) * 2 * 128 * kC * 4;
+constexpr size_t kScratchBytes = kOffPartLse + static_cast<size_t>(kNoAllocPairs) * 2 * 128 * 4;
+
+// ~8.5 MB on every device that loads the library, kept until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+struct DeviceSetup {
+  bool done = false;
+  unsigned char* scratch = nullptr;   // device address of g_noalloc_scratch on that device
+};
+DeviceSetup g_setup[64];
+std::mutex g_setup_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool cache_map(CUtensorMap* m, const void* base, uint64_t width, uint64_t rows, uint64_t batch,
+               int64_t stride_t, int64_t stride_b) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  cuuint64_t dims[3] = {width, rows, batch};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(stride_t) * 2, static_cast<cuuint64_t>(stride_b) * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kAttnKeysPerTile), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace mla
+
+using namespace mla;
+
+extern "C" mla_status mla_latent_attention_noalloc(
+    const void* q_abs, const int32_t* start_pos, int32_t rows, int32_t n_heads,
+    float softmax_scale, const void* kv_cache, int64_t kv_stride_b, int64_t kv_stride_t,
+    const void* pe_cache, int64_t pe_stride_b, int64_t pe_stride_t, int32_t max_seq_len,
+    void* o_lat, float* lse, int32_t* status, cudaStream_t stream) {
+  if (!q_abs || !start_pos || !kv_cache || !pe_cache || !o_lat) return MLA_ERR_INVALID_ARG;
+  if (rows < 1 || rows > kNoAllocMaxRows) return MLA_ERR_INVALID_ARG;   // beyond the scratch
+  if (n_heads < 16 || n_heads > 128 || n_heads % 16 != 0) return MLA_ERR_UNSUPPORTED;
+  if (max_seq_len < 64 || !(softmax_scale > 0.f)) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_abs) || !aligned16(o_lat) || !aligned16(kv_cache) || !aligned16(pe_cache) ||
+      (reinterpret_cast<uintptr_t>(start_pos) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+      (status && (reinterpret_cast<uintptr_t>(status) & 3u)))
+    return MLA_ERR_INVALID_ARG;
+  if (kv_stride_t < kC || pe_stride_t < kDr || kv_stride_b < 1 || pe_stride_b < 1 ||
+      (kv_stride_t * 2) % 16 || (pe_stride_t * 2) % 16 || (kv_stride_b * 2) % 16 ||
+      (pe_stride_b * 2) % 16)
+    return MLA_ERR_INVALID_ARG;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MLA_ERR_CUDA;
+  unsigned char* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_setup_mu);
+    DeviceSetup& su = g_setup[dev];
+    if (!su.done) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MLA_ERR_CUDA;
+      if (attention_prepare() != cudaSuccess) return MLA_ERR_CUDA;
+      su.scratch = static_cast<unsigned char*>(ptr);
+      su.done = true;
+    }
+    scratch = su.scratch;
+  }
+  int* st = status ? status : reinterpret_cast<int*>(scratch + kOffStatus);
+  long long* prefix = reinterpret_cast<long long*>(scratch + kOffPrefix);
+  float* part_o = reinterpret_cast<float*>(scratch + kOffPartO);
+  float* part_lse = reinterpret_cast<float*>(scratch + kOffPartLse);
+
+  CUtensorMap tm_kv, tm_pe;
+  if (!cache_map(&tm_kv, kv_cache, kC, max_seq_len, rows, kv_stride_t, kv_stride_b) ||
+      !cache_map(&tm_pe, pe_cache, kDr, max_seq_len, rows, pe_stride_t, pe_stride_b))
+    return MLA_ERR_INVALID_ARG;
+
+  // the internal status word starts at zero on every call; the prefix and partials are
+  // written before they are read within the call
+  if (!status && cudaMemsetAsync(st, 0, sizeof(int), stream) != cudaSuccess) return MLA_ERR_CUDA;
+
+  RmsParams rp{};
+  rp.rows = rows;
+  rp.T = 1;
+  rp.start_pos_dev = start_pos;
+  rp.max_seq_len = max_seq_len;
+  rp.row_prefix = prefix;
+  rp.status = st;
+  if (launch_key_prefix(rp, stream) != cudaSuccess) return MLA_ERR_CUDA;
+
+  const int pairs = attention_pairs() < kNoAllocPairs ? attention_pairs() : kNoAllocPairs;
+  AttnParams ap{};
+  ap.row_prefix = prefix;
+  ap.qabs = static_cast<const bf16*>(q_abs);
+  ap.rows = rows;
+  ap.T = 1;
+  ap.n_heads = n_heads;
+  ap.scale = softmax_scale;
+  ap.scale_log2 = softmax_scale * 1.4426950408889634f;
+  ap.min_keys_per_pair = 256;
+  ap.o_lat = static_cast<bf16*>(o_lat);
+  ap.lse_out = lse;
+  ap.max_seq_len = max_seq_len;
+  ap.part_o = part_o;
+  ap.part_lse = part_lse;
+  ap.status = st;
+  if (launch_attention(tm_kv, tm_pe, ap, pairs, stream) != cudaSuccess) return MLA_ERR_CUDA;
+
+  CombineParams cp{};
+  cp.row_prefix = prefix;
+  cp.rows = rows;
+  cp.n_heads = n_heads;
+  cp.n_pairs = pairs;
+  cp.min_keys_per_pair = 256;
+  cp.part_o = part_o;
+  cp.part_lse = part_lse;
+  cp.o_lat = static_cast<bf16*>(o_lat);
+  cp.lse_out = lse;
+  if (launch_combine(cp, stream) != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
+}

@@ -135,6 +135,33 @@ mla_status mla_prefill_chunk(mla_ctx* ctx, const void* q_latent, void* residual,
                              int64_t pe_stride_t, int32_t B, void* out, float* lse,
                              cudaStream_t stream);
 
+/* Latent attention without allocating memory (no counterpart on the source pages; an addition
+ * for callers that cannot allocate device memory where they run, e.g. code confined to a
+ * pre-reserved pool or given a fixed device budget by its host).
+ *
+ * Computes the attention step a5–a7 of mla_decode for caller-supplied absorbed queries:
+ *   q_abs [rows, 128, C+Dr] bf16 — per row the absorbed query q_lat ‖ q_pe of each head, heads
+ *     beyond n_heads padded with zeros (the layout mla_debug_copy(…, 2, …) returns);
+ *   start_pos [rows] int32 (device) — row r attends keys 0..start_pos[r] of cache sequence r;
+ *   caches and strides as for mla_decode, max_seq_len rows per sequence (>= 64);
+ *   o_lat [rows, n_heads, C] bf16 — softmax-weighted sum of cached latents;
+ *   lse [rows, n_heads] fp32 or NULL;
+ *   status — device int32 or NULL; device-side problems (a start position outside
+ *     [0, max_seq_len), a bounded wait that gave up) are recorded there (caller zeroes it).
+ * The library uses no memory but its inputs, its outputs and one fixed scratch array of about
+ * 8.5 MB that every device loading the library holds until exit.  Limits: rows <= 4096 (more
+ * returns MLA_ERR_INVALID_ARG); the split over keys uses at most 16 SM pairs.  The first call on
+ * a device sets the array up (address lookup, kernel attribute), so make it before capturing a
+ * stream into a graph.  All calls share the array: calls that can overlap on the GPU race and
+ * must be serialised by the caller. */
+mla_status mla_latent_attention_noalloc(const void* q_abs, const int32_t* start_pos,
+                                        int32_t rows, int32_t n_heads, float softmax_scale,
+                                        const void* kv_cache, int64_t kv_stride_b,
+                                        int64_t kv_stride_t, const void* pe_cache,
+                                        int64_t pe_stride_b, int64_t pe_stride_t,
+                                        int32_t max_seq_len, void* o_lat, float* lse,
+                                        int32_t* status, cudaStream_t stream);
+
 /* Synchronise `stream`, then read and clear the device status word of `ctx`: MLA_OK,
  * MLA_ERR_DEVICE_TIMEOUT or MLA_ERR_DEVICE_ARG (or MLA_ERR_CUDA if the synchronisation failed). */
 mla_status mla_sync_status(mla_ctx* ctx, cudaStream_t stream);
