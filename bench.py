@@ -69,6 +69,23 @@ def measured_peaks() -> dict:
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def profiled_traffic(workload_name: str):
+    """DRAM bytes (read + write) of one attention launch from the committed ncu summary, or None
+    when there is none for this workload or the kernel source changed since it was captured."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", f"latent_attention_{workload_name}.json")
+    src = os.path.join(ROOT, "head_latent_attention_11_b200", "csrc", "k_attn.cu")
+    if not (os.path.exists(prof) and os.path.exists(src)):
+        return None
+    with open(prof) as f:
+        d = json.load(f)
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if not sha.startswith(d.get("source_sha256_prefix", "-")):
+        return None
+    return int(d["dram_bytes_read"]) + int(d["dram_bytes_write"])
+
+
 # ------------------------------------------------------------------------------------------
 # Multi-rank aggregation (replicas: every rank runs its own batch, no data exchange)
 # ------------------------------------------------------------------------------------------
@@ -277,7 +294,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         achieved = work["attn_bytes"] / (attn_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": None, "kernel": "latent_attention",
+                "traffic": profiled_traffic(w.name), "kernel": "latent_attention",
                 "algorithmic_bytes_per_launch": work["attn_bytes"],
                 "peak_source": peaks["source"] + " (hbm_gbs, copy burst)"}
     else:
