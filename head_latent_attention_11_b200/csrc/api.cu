@@ -205,6 +205,9 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
       !make_map(&tm_pe, pe, kDr, c->cfg.max_seq_len, B, pe_st * 2, pe_sb * 2, 64, kAttnKeysPerTile, 1))
     return MLA_ERR_INVALID_ARG;
 
+  // Kernels 2-6 are launched with programmatic dependent launch: each starts on SMs its
+  // predecessor has released and waits (griddepcontrol.wait) before touching that kernel's data;
+  // kernel 1 is an ordinary launch, so the chain starts after all earlier work of the stream.
   // 1. q_norm (+ residual), rotary table, key prefix
   RmsParams rp{};
   rp.x = static_cast<const bf16*>(q_latent);
@@ -239,7 +242,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   g1.n_heads = H;
   g1.status = c->status();
   clk.mark("wq_b_rope");
-  MLA_TRY(launch_gemm(c->tm_wq, tm_y, g1, 1, s));
+  MLA_TRY(launch_gemm(c->tm_wq, tm_y, g1, 1, s, true));
   ++launches;
 
   // 3. W_UK absorption (one batch per head)
@@ -254,7 +257,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   g2.n_heads = H;
   g2.status = c->status();
   clk.mark("absorb_w_uk");
-  MLA_TRY(launch_gemm(c->tm_wukt, tm_qn, g2, H, s));
+  MLA_TRY(launch_gemm(c->tm_wukt, tm_qn, g2, H, s, true));
   ++launches;
 
   // 4. latent attention
@@ -275,7 +278,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   ap.part_lse = c->part_lse();
   ap.status = c->status();
   clk.mark("latent_attention");
-  MLA_TRY(launch_attention(tm_kv, tm_pe, ap, c->n_pairs, s));
+  MLA_TRY(launch_attention(tm_kv, tm_pe, ap, c->n_pairs, s, true));
   ++launches;
 
   // 5. combine rows cut between pairs
@@ -290,7 +293,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   cp.o_lat = c->o_lat();
   cp.lse_out = lse;
   clk.mark("combine");
-  MLA_TRY(launch_combine(cp, s));
+  MLA_TRY(launch_combine(cp, s, true));
   ++launches;
 
   // 6. W_UV expansion (one batch per head)
@@ -306,7 +309,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   g3.n_heads = H;
   g3.status = c->status();
   clk.mark("w_uv");
-  MLA_TRY(launch_gemm(c->tm_wuv, tm_olat, g3, H, s));
+  MLA_TRY(launch_gemm(c->tm_wuv, tm_olat, g3, H, s, true));
   ++launches;
   clk.finish();
 

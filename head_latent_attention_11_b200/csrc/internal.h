@@ -100,14 +100,33 @@ struct CombineParams {
   float* lse_out;
 };
 
-// Launchers (defined next to their kernels).
+// Launch configuration; with pdl set the kernel is launched with programmatic stream
+// serialisation: its CTAs may start while the previous kernel of the stream is still running, and
+// it waits (griddepcontrol.wait) before it reads or writes anything that kernel touches.
+struct LaunchCfg {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  LaunchCfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl) {
+    cfg = cudaLaunchConfig_t{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+  }
+};
+
+// Launchers (defined next to their kernels).  pdl: see LaunchCfg.
 cudaError_t launch_rmsnorm(const RmsParams& p, cudaStream_t s);
 cudaError_t launch_key_prefix(const RmsParams& p, cudaStream_t s);   // row_prefix only
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
-                        int batches, cudaStream_t s);
+                        int batches, cudaStream_t s, bool pdl);
 cudaError_t launch_attention(const CUtensorMap& tkv, const CUtensorMap& tpe, const AttnParams& p,
-                             int n_pairs, cudaStream_t s);
-cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
+                             int n_pairs, cudaStream_t s, bool pdl);
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t s, bool pdl);
 cudaError_t launch_transpose_uk(const bf16* wkv_b, bf16* w_ukt, int n_heads, cudaStream_t s);
 cudaError_t gemm_prepare();        // one-time per-device attribute set-up
 cudaError_t attention_prepare();

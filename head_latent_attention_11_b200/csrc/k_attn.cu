@@ -140,6 +140,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   float* sRed = reinterpret_cast<float*>(smem + kOffRed);   // m_ref, seq, 2 x row sums
   Bars* bar = reinterpret_cast<Bars*>(smem + kOffBar);
 
+  pdl_launch_dependents();
+  pdl_wait();   // queries, key prefix and status come from the kernels before this one
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int pair = static_cast<int>(cluster_id_x());
@@ -595,9 +597,9 @@ cudaError_t attention_prepare() {
 }
 
 cudaError_t launch_attention(const CUtensorMap& tkv, const CUtensorMap& tpe, const AttnParams& p,
-                             int n_pairs, cudaStream_t s) {
-  latent_attention_kernel<<<dim3(2 * n_pairs), dim3(kThreads), kAttnSmem, s>>>(tkv, tpe, p);
-  return cudaGetLastError();
+                             int n_pairs, cudaStream_t s, bool pdl) {
+  LaunchCfg lc(dim3(2 * n_pairs), dim3(kThreads), kAttnSmem, s, pdl);
+  return cudaLaunchKernelEx(&lc.cfg, latent_attention_kernel, tkv, tpe, p);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -613,6 +615,8 @@ __device__ __forceinline__ int pair_of_key(long long total, int pairs, long long
 }
 
 __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int r = blockIdx.x;
   const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -650,9 +654,9 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   if (lane == 0 && p.lse_out) p.lse_out[static_cast<size_t>(r) * p.n_heads + h] = mx + logf(wsum);
 }
 
-cudaError_t launch_combine(const CombineParams& p, cudaStream_t s) {
-  combine_kernel<<<dim3(p.rows, (p.n_heads + 3) / 4), 128, 0, s>>>(p);
-  return cudaGetLastError();
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t s, bool pdl) {
+  LaunchCfg lc(dim3(p.rows, (p.n_heads + 3) / 4), dim3(128), 0, s, pdl);
+  return cudaLaunchKernelEx(&lc.cfg, combine_kernel, p);
 }
 
 }  // namespace mla

@@ -7,15 +7,19 @@
 // wkv_b[:, :nope] ("bshd,hdc->bshc") and the attention result expanded through wkv_b[:, -v:]
 // ("bshc,hdc->bshd").
 //
-// All three are "weights as M" GEMMs: A is a weight matrix (128 weight rows per CTA, K-major),
+// All three are "weights as M" GEMMs: A is a weight matrix (128 weight rows per tile, K-major),
 // B holds the token rows (K-major), so decode batches of a few tokens still fill the 128-row MMA.
-// One CTA computes one 128 x BN output tile of one batch g (= head for a4/a8):
+// The kernel is persistent: one CTA per SM walks the output tiles ("units": batch g = head for
+// a4/a8, 128-row weight tile, BN-token tile) round-robin, and its TMA ring streams K slabs
+// continuously across unit boundaries, so weight streaming never drains between tiles.
 //   warp 0      TMA producer: 64-wide K slabs of A (128 x 64) and B (BN x 64), 128-byte swizzle,
-//               into a STAGES-deep shared-memory ring;
-//   warp 1      allocates TMEM and issues tcgen05.mma (M=128, N=BN, K=16) per slab, committing
-//               each slab back to the producer and the finished tile to the epilogue;
+//               into a STAGES-deep shared-memory ring (~200 KB, one CTA per SM);
+//   warp 1      allocates TMEM and issues tcgen05.mma (M=128, N=BN, K=16) per slab into one of
+//               two accumulators (units alternate), committing each slab back to the producer
+//               and each finished unit to the epilogue;
 //   warps 2-5   epilogue: tcgen05.ld the fp32 accumulator (thread = weight row), apply RoPE for
-//               the rotary rows of wq_b (partner of a pair = neighbouring lane), store bf16.
+//               the rotary rows of wq_b (partner of a pair = neighbouring lane), store bf16,
+//               hand the accumulator back — overlapping the next unit's MMAs.
 #include "internal.h"
 #include "tc100.cuh"
 
@@ -29,7 +33,7 @@ constexpr int kSlabA = 128 * 64 * 2;   // 16 KB
 template <int BN>
 struct GemmTile {
   static constexpr int kSlabB = BN * 64 * 2;
-  static constexpr int kTmemCols = BN < 32 ? 32 : BN;
+  static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;   // two accumulators
 };
 
 template <int BN, int STAGES>
@@ -38,7 +42,7 @@ constexpr int gemm_smem_bytes() {
 }
 
 __device__ __forceinline__ void epi_store(const GemmParams& p, int g, int m, int n, float v,
-                                          float partner, bool rope_row, int rope_j) {
+                                          float partner) {
   if (p.epi == kEpiWqbRope) {
     const int h = m / kDq, j = m - h * kDq;
     if (j < kDn) {
@@ -61,10 +65,41 @@ __device__ __forceinline__ void epi_store(const GemmParams& p, int g, int m, int
   }
 }
 
+struct Unit {
+  int g, m0, n0;
+};
+
+__device__ __forceinline__ Unit unit_of(int u, int mt, int nt, int BN) {
+  // tokens fastest: consecutive units share a weight tile (its re-reads hit L2)
+  Unit r;
+  const int n = u % nt;
+  const int rest = u / nt;
+  r.m0 = (rest % mt) * 128;
+  r.g = rest / mt;
+  r.n0 = n * BN;
+  return r;
+}
+
+// Work split: CTA c takes units c, c + G, c + 2G, ... (G = grid size).
+struct Sched {
+  int units, G, u;
+  __device__ void init(int nunits, int grid, int cta) {
+    units = nunits;
+    G = grid;
+    u = cta;
+  }
+  __device__ bool next(int& unit) {
+    if (u >= units) return false;
+    unit = u;
+    u += G;
+    return true;
+  }
+};
+
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const GemmParams p) {
+                     const GemmParams p, const int batches) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -73,23 +108,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * GemmTile<BN>::kSlabB);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
-  uint64_t* dfull = bars + 2 * STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  uint64_t* acc_full = bars + 2 * STAGES;        // [2]
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;   // [2]
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  pdl_launch_dependents();
   const int warp = warp_id();
-  const int m0 = blockIdx.x * 128;
-  const int n0 = blockIdx.y * BN;
-  const int g = blockIdx.z;
   const int nk = p.K / 64;
+  const int mt = p.M / 128;
+  const int nt = (p.N + BN - 1) / BN;
+  const int total = batches * mt * nt;
   Guard guard{abort_flag, p.status};
+  Sched sched;
+  sched.init(total, gridDim.x, blockIdx.x);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(dfull, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -103,90 +147,143 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     if (elect_one()) {
-      int issued = 0;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % STAGES;
-        if (kb >= STAGES && !mbar_wait(&empty[s], ((kb / STAGES) - 1) & 1, guard)) break;
-        mbar_arrive_expect_tx(&full[s], kSlabA + GemmTile<BN>::kSlabB);
-        tma_load_3d(sA + s * kSlabA, &tmA, &full[s], kb * 64, m0 + p.a_row_off, g);
-        tma_load_3d(sB + s * GemmTile<BN>::kSlabB, &tmB, &full[s], kb * 64, g, n0);
-        ++issued;
+      const uint64_t pol_w = policy_evict_first();   // weights are read once per call
+      // The weight slabs of the first ring pass do not depend on the previous kernel: issue them
+      // before waiting for it, so weight streaming overlaps that kernel's tail.
+      int npre = 0;
+      {
+        Sched pre = sched;
+        int u;
+        while (npre < STAGES && pre.next(u)) {
+          const Unit un = unit_of(u, mt, nt, BN);
+          for (int j = 0; j < nk && npre < STAGES; ++j, ++npre) {
+            mbar_arrive_expect_tx(&full[npre], kSlabA + GemmTile<BN>::kSlabB);
+            tma_load_3d_hint(sA + npre * kSlabA, &tmA, &full[npre], j * 64, un.m0 + p.a_row_off,
+                             un.g, pol_w);
+          }
+        }
+      }
+      pdl_wait();
+      int ks = 0;
+      bool ok = true;
+      int u;
+      while (ok && sched.next(u)) {
+        const Unit un = unit_of(u, mt, nt, BN);
+        for (int j = 0; j < nk; ++j, ++ks) {
+          const int s = ks % STAGES;
+          if (ks >= npre) {
+            if (ks >= STAGES && !mbar_wait(&empty[s], ((ks / STAGES) - 1) & 1, guard)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[s], kSlabA + GemmTile<BN>::kSlabB);
+            tma_load_3d_hint(sA + s * kSlabA, &tmA, &full[s], j * 64, un.m0 + p.a_row_off, un.g,
+                             pol_w);
+          }
+          tma_load_3d(sB + s * GemmTile<BN>::kSlabB, &tmB, &full[s], j * 64, un.g, un.n0);
+        }
       }
       if (guard.aborted()) {
         // drain the loads still in flight before the CTA's shared memory goes away
         int dummy = 0;
-        Guard drain{reinterpret_cast<volatile int*>(&dummy), p.status};
-        for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb)
-          mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, drain);
+        Guard dr{reinterpret_cast<volatile int*>(&dummy), p.status};
+        for (int k = ks > STAGES ? ks - STAGES : 0; k < ks; ++k)
+          mbar_wait(&full[k % STAGES], (k / STAGES) & 1, dr);
       }
     }
   } else if (warp == 1) {
     if (elect_one()) {
       const uint32_t idesc = idesc_bf16(128, BN, false, false);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % STAGES;
-        if (!mbar_wait(&full[s], (kb / STAGES) & 1, guard)) break;
+      int ks = 0, si = 0;
+      bool ok = true;
+      int u;
+      while (ok && sched.next(u)) {
+        const int ab = si & 1;
+        if (si >= 2 && !mbar_wait(&acc_empty[ab], ((si >> 1) - 1) & 1, guard)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + s * kSlabA);
-        const uint32_t b0 = smem_u32(sB + s * GemmTile<BN>::kSlabB);
+        const uint32_t d = tmem + ab * BN;
+        for (int j = 0; j < nk; ++j, ++ks) {
+          const int s = ks % STAGES;
+          if (!mbar_wait(&full[s], (ks / STAGES) & 1, guard)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kSlabA);
+          const uint32_t b0 = smem_u32(sB + s * GemmTile<BN>::kSlabB);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          umma_bf16(tmem, smem_desc_sw128(a0 + kk * 32, 16, 1024),
-                    smem_desc_sw128(b0 + kk * 32, 16, 1024), idesc, (kb | kk) != 0);
+          for (int kk = 0; kk < 4; ++kk) {
+            umma_bf16(d, smem_desc_sw128(a0 + kk * 32, 16, 1024),
+                      smem_desc_sw128(b0 + kk * 32, 16, 1024), idesc, (j | kk) != 0);
+          }
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[s]);
+        if (!ok) break;
+        umma_commit(&acc_full[ab]);
+        ++si;
       }
-      umma_commit(dfull);
+      umma_commit(drain);
     }
   } else {
     // epilogue warps 2..5 → TMEM lane quadrant warp % 4
+    pdl_wait();   // outputs may be read by the kernel before this one
     const int quad = warp & 3;
     const int row = quad * 32 + static_cast<int>(lane_id());
-    const int m = m0 + row;
-    const bool ok = warp_wait(dfull, 0, guard);   // converged warp for tcgen05.ld
-    tc_fence_after();
-    if (ok) {
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-      const bool rope_row = (p.epi == kEpiWqbRope) && ((m % kDq) >= kDn);
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    int si = 0;
+    int u;
+    while (sched.next(u)) {
+      const Unit un = unit_of(u, mt, nt, BN);
+      const int ab = si & 1;
+      if (!warp_wait(&acc_full[ab], (si >> 1) & 1, guard)) break;
+      tc_fence_after();
+      const int m = un.m0 + row;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 16) {
+        if (un.n0 + c0 >= p.N) break;   // uniform across the warp
         float v[16];
-        tmem_ld16(taddr + c0, v);
+        tmem_ld16(tmem + lane_off + ab * BN + c0, v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float partner = __shfl_xor_sync(0xffffffffu, v[i], 1);
-          const int n = n0 + c0 + i;
-          if (n < p.N) epi_store(p, g, m, n, v[i], partner, rope_row, 0);
+          const int n = un.n0 + c0 + i;
+          if (n < p.N) epi_store(p, un.g, m, n, v[i], partner);
         }
       }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
+      ++si;
     }
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    if (guard.aborted()) {
-      // make sure no MMA still writes the accumulator before it is released
-      int dummy = 0;
-      Guard drain{reinterpret_cast<volatile int*>(&dummy), p.status};
-      mbar_wait(dfull, 0, drain);
-    }
+    int dummy = 0;
+    Guard dr{reinterpret_cast<volatile int*>(&dummy), p.status};
+    mbar_wait(drain, 0, dr);   // no MMA still writes the accumulators
     tc_fence_after();
     tmem_dealloc(tmem, GemmTile<BN>::kTmemCols);
   }
 }
 
+int g_num_sms = 0;
+
 template <int BN, int STAGES>
 cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
-                          int batches, cudaStream_t s) {
-  dim3 grid(p.M / 128, (p.N + BN - 1) / BN, batches);
-  gemm_bf16_kernel<BN, STAGES>
-      <<<grid, kGemmThreads, gemm_smem_bytes<BN, STAGES>(), s>>>(ta, tb, p);
-  return cudaGetLastError();
+                          int batches, cudaStream_t s, bool pdl) {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 1;
+  }
+  const int total = batches * (p.M / 128) * ((p.N + BN - 1) / BN);
+  const int grid = total < g_num_sms ? total : g_num_sms;
+  LaunchCfg lc(dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<BN, STAGES>(), s, pdl);
+  return cudaLaunchKernelEx(&lc.cfg, gemm_bf16_kernel<BN, STAGES>, ta, tb, p, batches);
 }
 
 template <int BN, int STAGES>
 cudaError_t set_attr() {
+  static_assert(gemm_smem_bytes<BN, STAGES>() <= 232448, "shared memory budget");
   return cudaFuncSetAttribute(gemm_bf16_kernel<BN, STAGES>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               gemm_smem_bytes<BN, STAGES>());
@@ -194,21 +291,20 @@ cudaError_t set_attr() {
 
 }  // namespace
 
-// Tile choice: BN covers the token count up to 256; decode tiles keep several CTAs per SM
-// resident (small rings, small TMEM), the 256-wide prefill tile uses one CTA per SM.
+// Tile choice: BN covers the token count up to 256; the ring fills ~200 KB of shared memory.
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
-                        int batches, cudaStream_t s) {
-  if (p.N <= 32) return launch_gemm_t<32, 5>(ta, tb, p, batches, s);
-  if (p.N <= 64) return launch_gemm_t<64, 4>(ta, tb, p, batches, s);
-  if (p.N <= 128) return launch_gemm_t<128, 4>(ta, tb, p, batches, s);
-  return launch_gemm_t<256, 4>(ta, tb, p, batches, s);
+                        int batches, cudaStream_t s, bool pdl) {
+  if (p.N <= 32) return launch_gemm_t<32, 10>(ta, tb, p, batches, s, pdl);
+  if (p.N <= 64) return launch_gemm_t<64, 8>(ta, tb, p, batches, s, pdl);
+  if (p.N <= 128) return launch_gemm_t<128, 6>(ta, tb, p, batches, s, pdl);
+  return launch_gemm_t<256, 4>(ta, tb, p, batches, s, pdl);
 }
 
 cudaError_t gemm_prepare() {
   cudaError_t e;
-  if ((e = set_attr<32, 5>()) != cudaSuccess) return e;
-  if ((e = set_attr<64, 4>()) != cudaSuccess) return e;
-  if ((e = set_attr<128, 4>()) != cudaSuccess) return e;
+  if ((e = set_attr<32, 10>()) != cudaSuccess) return e;
+  if ((e = set_attr<64, 8>()) != cudaSuccess) return e;
+  if ((e = set_attr<128, 6>()) != cudaSuccess) return e;
   return set_attr<256, 4>();
 }
 

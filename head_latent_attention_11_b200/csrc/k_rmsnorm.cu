@@ -61,6 +61,7 @@ __device__ void key_prefix_block(const RmsParams& p) {
 
 template <int NCH>
 __global__ void __launch_bounds__(128) rmsnorm_kernel(const RmsParams p) {
+  pdl_launch_dependents();   // the wq_b GEMM may start streaming its weight now
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 4 + warp;
   if (row < p.rows) {

@@ -147,7 +147,7 @@ extern "C" mla_status mla_latent_attention_noalloc(
   ap.part_o = part_o;
   ap.part_lse = part_lse;
   ap.status = st;
-  if (launch_attention(tm_kv, tm_pe, ap, pairs, stream) != cudaSuccess) return MLA_ERR_CUDA;
+  if (launch_attention(tm_kv, tm_pe, ap, pairs, stream, false) != cudaSuccess) return MLA_ERR_CUDA;
 
   CombineParams cp{};
   cp.row_prefix = prefix;
@@ -159,6 +159,6 @@ extern "C" mla_status mla_latent_attention_noalloc(
   cp.part_lse = part_lse;
   cp.o_lat = static_cast<bf16*>(o_lat);
   cp.lse_out = lse;
-  if (launch_combine(cp, stream) != cudaSuccess) return MLA_ERR_CUDA;
+  if (launch_combine(cp, stream, false) != cudaSuccess) return MLA_ERR_CUDA;
   return MLA_OK;
 }

@@ -43,6 +43,14 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
+// Programmatic dependent launch.  launch_dependents lets the next kernel of the stream start its
+// CTAs (on free SMs) before this one ends; wait blocks until every kernel this one depends on has
+// completed and its memory writes are visible.  Both are no-ops for a kernel launched normally.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------------------------------
 // Abort / status plumbing shared by the warps of one CTA
 // ------------------------------------------------------------------------------------------
