@@ -3,7 +3,9 @@
 One step = one full decode call (q_norm → wq_b+RoPE → W_UK absorption → latent attention over
 the cache → combine → W_UV) for the DeepSeek-V3.2-shaped decode batch: B=32 sequences, H=128,
 cache L=4096 (keys 0..4096), bf16, synthetic seeded inputs resident in HBM.  Between timed steps
-L2 is flushed by writing a 256 MiB buffer (the step's own inputs are 261 MB as well).
+L2 is flushed by writing a 256 MiB buffer and then reading another 256 MiB buffer (both untimed):
+the step starts with none of its data in L2, and without 126 MB of dirty flush lines that the
+step's own loads and stores would otherwise have to write back (the step's inputs are 261 MB).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
         [--workload v32_decode|kimi_decode|ragged_decode|tiny_decode|prefill_chunk]
@@ -197,7 +199,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     out_shape = (B, H, 128) if w.mode == "decode" else (B, T, H, 128)
     out = torch.empty(out_shape, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+
+    def flush_l2(i: int) -> None:
+        flush.fill_(float(i))   # evict everything the previous step left in L2 ...
+        flush_rd.sum()          # ... and leave L2 holding clean lines of an unrelated buffer
 
     def step():
         if w.mode == "decode":
@@ -221,7 +228,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     clocks.start()
     time.sleep(0.3)
     for i in range(args.steps):
-        flush.fill_(float(i))
+        flush_l2(i)
         starts[i].record(stream)
         step()
         ends[i].record(stream)
@@ -239,7 +246,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     mla_enable_stage_timing(rt.ctx, True)
     stage_acc: dict[str, list[float]] = {}
     for i in range(max(3, min(args.steps, 20))):
-        flush.fill_(float(i))
+        flush_l2(i)
         step()
         for name, ms in mla_stage_times(rt.ctx):
             stage_acc.setdefault(name, []).append(ms)
@@ -256,7 +263,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     d_sp = torch.empty_like(start_pos)
     e2e_ms = []
     for i in range(args.steps):
-        flush.fill_(float(i))
+        flush_l2(i)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         d_q.copy_(h_q, non_blocking=True)
@@ -313,7 +320,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         "config": {"workload": w.name, "batch": B, "tokens": T, "n_heads": H,
                    "cache_keys_per_step": work["keys"], "q_lora": 1536, "kv_lora": 512,
                    "rope": 64, "v": 128,
-                   "l2": "flushed before every timed step (256 MiB write, untimed)",
+                   "l2": "flushed before every timed step: 256 MiB write, then 256 MiB read of another buffer (untimed)",
                    "parallelism": f"replicas x{world} (sequence-sharded, no collective)"},
         "hbm": {"step_bytes": work["bytes"], "step_gbs": round(step_gbs, 1),
                 "frac_of_peak": round(step_gbs / peaks["hbm_gbs"], 4)},

@@ -43,6 +43,28 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+}  // namespace
+
+bool mla::encode_tiled(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
+                  const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+                  CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rank < 1 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) st[i] = strides[i];
+  }
+  return fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, b, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
 // 3-D bf16 tensor map with 128-byte swizzle; strides in bytes for dims 1 and 2.
 bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
               uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
@@ -62,7 +84,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
-  size_t status, w_ukt, y, rope, q_nope, qabs, o_lat, part_o, part_lse, prefix, total;
+  size_t status, w_ukt, y, rope, q_nope, qabs, o_lat, part_o, part_lse, prefix, pair_row, total;
 };
 
 int device_pairs() { return attention_pairs(); }
@@ -106,6 +128,7 @@ Layout layout_of(const mla_config* c) {
   L.part_o = take(pairs * 2 * 128 * kC * 4);
   L.part_lse = take(pairs * 2 * 128 * 4);
   L.prefix = take((rows + 1) * 8);
+  L.pair_row = take(pairs * 4);
   L.total = off;
   return L;
 }
@@ -140,6 +163,7 @@ struct mla_ctx {
   float* part_o() const { return reinterpret_cast<float*>(ws + L.part_o); }
   float* part_lse() const { return reinterpret_cast<float*>(ws + L.part_lse); }
   long long* prefix() const { return reinterpret_cast<long long*>(ws + L.prefix); }
+  int* pair_row() const { return reinterpret_cast<int*>(ws + L.pair_row); }
 };
 
 namespace {
@@ -194,15 +218,16 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   int launches = 0;
 
   // per-call tensor maps
-  CUtensorMap tm_y, tm_qn, tm_olat, tm_kv, tm_pe;
+  CUtensorMap tm_y, tm_qn, tm_olat;
+  AttnMaps am;
   const uint64_t rws = static_cast<uint64_t>(rows);
   if (!make_map(&tm_y, c->y(), kR, 1, rws, kR * 2, kR * 2, 64, 1, bn) ||
       !make_map(&tm_qn, c->q_nope(), kDn, H, rws, kDn * 2, static_cast<uint64_t>(H) * kDn * 2, 64,
                 1, bn) ||
       !make_map(&tm_olat, c->o_lat(), kC, H, rws, kC * 2, static_cast<uint64_t>(H) * kC * 2, 64, 1,
                 bn) ||
-      !make_map(&tm_kv, kv, kC, c->cfg.max_seq_len, B, kv_st * 2, kv_sb * 2, 64, kAttnKeysPerTile, 1) ||
-      !make_map(&tm_pe, pe, kDr, c->cfg.max_seq_len, B, pe_st * 2, pe_sb * 2, 64, kAttnKeysPerTile, 1))
+      !make_attention_maps(&am, kv, kv_sb, kv_st, pe, pe_sb, pe_st, B, c->cfg.max_seq_len, c->qabs(),
+                           rows, c->o_lat(), H, c->part_o(), c->n_pairs))
     return MLA_ERR_INVALID_ARG;
 
   // Kernels 2-6 are launched with programmatic dependent launch: each starts on SMs its
@@ -224,6 +249,9 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   rp.T = T;
   rp.max_seq_len = c->cfg.max_seq_len;
   rp.row_prefix = c->prefix();
+  rp.pair_row = c->pair_row();
+  rp.n_pairs = c->n_pairs;
+  rp.min_keys_per_pair = kMinKeysPerPair;
   rp.status = c->status();
   clk.mark("rmsnorm");
   MLA_TRY(launch_rmsnorm(rp, s));
@@ -276,9 +304,10 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   ap.max_seq_len = c->cfg.max_seq_len;
   ap.part_o = c->part_o();
   ap.part_lse = c->part_lse();
+  ap.pair_row = c->pair_row();
   ap.status = c->status();
   clk.mark("latent_attention");
-  MLA_TRY(launch_attention(tm_kv, tm_pe, ap, c->n_pairs, s, true));
+  MLA_TRY(launch_attention(am, ap, c->n_pairs, s, true));
   ++launches;
 
   // 5. combine rows cut between pairs

@@ -43,6 +43,11 @@ struct RmsParams {
   int max_seq_len;
   // key prefix over rows (written by block 0); null to skip
   long long* row_prefix;    // [rows + 1]
+  // first row of each attention pair's key range (written by block 0 after the prefix);
+  // null to skip.  n_pairs / min_keys_per_pair as given to the attention kernel.
+  int* pair_row;            // [n_pairs]
+  int n_pairs;
+  int min_keys_per_pair;
   int* status;
 };
 
@@ -85,6 +90,7 @@ struct AttnParams {
   int max_seq_len;
   float* part_o;                // [pairs, 2, 128, 512] fp32 normalised partial outputs
   float* part_lse;              // [pairs, 2, 128]
+  const int* pair_row;          // [pairs] first row of each pair's key range, or null
   int* status;
 };
 
@@ -99,6 +105,12 @@ struct CombineParams {
   bf16* o_lat;
   float* lse_out;
 };
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no interleave, L2 256-byte
+// promotion, zero fill).  dims/box have `rank` entries, strides (bytes) rank - 1.
+bool encode_tiled(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
+                  const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+                  CUtensorMapSwizzle swizzle);
 
 // Launch configuration; with pdl set the kernel is launched with programmatic stream
 // serialisation: its CTAs may start while the previous kernel of the stream is still running, and
@@ -124,8 +136,20 @@ cudaError_t launch_rmsnorm(const RmsParams& p, cudaStream_t s);
 cudaError_t launch_key_prefix(const RmsParams& p, cudaStream_t s);   // row_prefix only
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                         int batches, cudaStream_t s, bool pdl);
-cudaError_t launch_attention(const CUtensorMap& tkv, const CUtensorMap& tpe, const AttnParams& p,
-                             int n_pairs, cudaStream_t s, bool pdl);
+// Tensor maps of the attention kernel, built on the host for each call (all 128-byte swizzle).
+struct AttnMaps {
+  CUtensorMap kv;    // latent cache  bf16 {512, max_seq_len, batch}, box {64, 32, 1}
+  CUtensorMap pe;    // rotary cache  bf16 {64, max_seq_len, batch},  box {64, 32, 1}
+  CUtensorMap q;     // absorbed queries bf16 {576, 128, rows},       box {64, 128, 1}
+  CUtensorMap o;     // o_lat         bf16 {512, n_heads, rows},      box {64, 32, 1}
+  CUtensorMap part;  // split partials fp32 {512, pairs * 2 * 128},   box {32, 32}
+};
+// Strides in elements; false if a map cannot be encoded (alignment, sizes).
+bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,
+                         int64_t pe_sb, int64_t pe_st, int batch, int max_seq_len, const void* qabs,
+                         int rows, const void* o_lat, int n_heads, const void* part_o, int pairs);
+cudaError_t launch_attention(const AttnMaps& m, const AttnParams& p, int n_pairs, cudaStream_t s,
+                             bool pdl);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s, bool pdl);
 cudaError_t launch_transpose_uk(const bf16* wkv_b, bf16* w_ukt, int n_heads, cudaStream_t s);
 cudaError_t gemm_prepare();        // one-time per-device attribute set-up
@@ -145,6 +169,18 @@ __host__ __device__ inline int active_pairs(long long total_keys, int launched, 
 }
 __host__ __device__ inline long long pair_begin(long long total_keys, int pairs, int p) {
   return total_keys * p / pairs;
+}
+
+// Row containing flattened key e: largest r with prefix[r] <= e (plain loads: the prefix may
+// have been written earlier by the calling kernel).
+__device__ __forceinline__ int row_of_key(const long long* prefix, int rows, long long e) {
+  int lo = 0, hi = rows - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= e) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
 }
 
 }  // namespace mla

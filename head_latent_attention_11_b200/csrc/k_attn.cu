@@ -29,7 +29,9 @@
 //     group one thread owns one head row.  Only the running-max decision is handed from tile to
 //     tile across the groups (per-row flag in shared memory); each group keeps its own partial
 //     row sum, so the softmax work of consecutive tiles overlaps.
-//   * Each warp stages its 32 rows of partial scores and ships them with its own 4 KB bulk copy.
+//   * Each warp stages its 32 rows of partial scores and ships them with its own 4 KB bulk copy;
+//     it waits only for the copy of its counterpart warp (same group and lane quarter) in the
+//     peer CTA, through a barrier pair of its own.
 //   * The flattened key range of all rows is split evenly over the cluster pairs (split-K over
 //     keys, also across row boundaries); a row cut between pairs leaves normalised partials
 //     (O/l, lse) for the combine kernel, an uncut row is written as bf16 o_lat directly.
@@ -48,8 +50,10 @@ namespace {
 
 constexpr int kNK = kAttnKeysPerTile;      // keys per tile
 constexpr int kStages = 7;                 // cache tile ring depth
+constexpr int kL2Ahead = 12;               // tiles the L2 prefetch runs ahead of the ring loads
 constexpr int kSlabKV = kNK * 128;         // 4 KB: 64 columns x 32 keys, bf16
 constexpr int kMaxSlabs = 5;               // rank 1: 4 latent slabs + 1 rotary slab
+constexpr int kSlabQ = 128 * 64 * 2;       // 16 KB: 64 query columns of all 128 head rows
 constexpr int kStageBytes = kMaxSlabs * kSlabKV;
 constexpr int kXSlot = 128 * kNK * 4;      // 16 KB: one partial score tile, fp32
 
@@ -73,10 +77,10 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t q_full, q_empty;
+  uint64_t q_empty;         // the piece's last score MMA has read the query in TMEM
   uint64_t s_full[6], p_full[kNS], pv_done[6];
   uint64_t o_empty;
-  uint64_t x_full[2], x_empty[2];
+  uint64_t x_full[8], x_empty[8];   // [group][warp quad]
   uint64_t sync_all;       // the 256 softmax threads
   uint64_t drain;
   uint32_t tmem_slot;
@@ -85,29 +89,19 @@ struct Bars {
 static_assert(sizeof(Bars) <= 512, "barrier block");
 static_assert(kAttnSmem <= 232448, "shared memory budget");
 
-// Row containing flattened key e: largest r with prefix[r] <= e.
-__device__ __forceinline__ int row_of_key(const long long* prefix, int rows, long long e) {
-  int lo = 0, hi = rows - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(prefix + mid) <= e) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
-}
-
 // Iterates the pieces (row, [k0, k1)) of one pair's key range.
 struct PieceIter {
   const long long* prefix;
   int rows;
   long long e0, e1;
   int r;
-  __device__ void init(const long long* pf, int nrows, long long b, long long e) {
+  // first_row: the row containing key b when known (else -1: binary search)
+  __device__ void init(const long long* pf, int nrows, long long b, long long e, int first_row) {
     prefix = pf;
     rows = nrows;
     e0 = b;
     e1 = e;
-    r = row_of_key(pf, nrows, b);
+    r = first_row >= 0 ? first_row : row_of_key(pf, nrows, b);
   }
   __device__ bool get(int& row, int& k0, int& k1, int& nkeys_row, bool& first_row) const {
     if (r >= rows) return false;
@@ -130,7 +124,10 @@ __device__ __forceinline__ uint32_t xbuf_off(int slot, int h, int c) {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     latent_attention_kernel(const __grid_constant__ CUtensorMap tmKV,
-                            const __grid_constant__ CUtensorMap tmPE, const AttnParams p) {
+                            const __grid_constant__ CUtensorMap tmPE,
+                            const __grid_constant__ CUtensorMap tmQ,
+                            const __grid_constant__ CUtensorMap tmO,
+                            const __grid_constant__ CUtensorMap tmPart, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -140,15 +137,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   float* sRed = reinterpret_cast<float*>(smem + kOffRed);   // m_ref, seq, 2 x row sums
   Bars* bar = reinterpret_cast<Bars*>(smem + kOffBar);
 
+  // Programmatic dependent launch: the key prefix is final before this kernel can start (the
+  // RMSNorm kernel publishes it before releasing its dependents) and the cache is an input of the
+  // whole chain, so the producer streams cache tiles right away; the warps that read queries or
+  // write outputs wait for the previous kernels first.
   pdl_launch_dependents();
-  pdl_wait();   // queries, key prefix and status come from the kernels before this one
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int pair = static_cast<int>(cluster_id_x());
   const int launched_pairs = static_cast<int>(nclusters_x());
   const long long total = __ldg(p.row_prefix + p.rows);
+  const int row0 = p.pair_row ? __ldg(p.pair_row + pair) : -1;   // same round trip as total
   const int pairs = active_pairs(total, launched_pairs, p.min_keys_per_pair);
-  if (pair >= pairs) return;   // both CTAs of the pair take this branch together
+  if (pair >= pairs) {         // both CTAs of the pair take this branch together
+    pdl_wait();
+    return;
+  }
   const long long e0 = pair_begin(total, pairs, pair), e1 = pair_begin(total, pairs, pair + 1);
 
   const int warp = static_cast<int>(warp_id());
@@ -161,16 +165,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&bar->kv_full[i], 1);
       mbar_init(&bar->kv_empty[i], 1);
     }
-    mbar_init(&bar->q_full, kSoftmaxThreads);
     mbar_init(&bar->q_empty, 1);
     for (int i = 0; i < 6; ++i) {
       mbar_init(&bar->s_full[i], 1);
       mbar_init(&bar->pv_done[i], 1);
     }
     for (int i = 0; i < kNS; ++i) mbar_init(&bar->p_full[i], 128);   // the tile's group
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar->x_full[i], 1);     // receiver's expect_tx + the peer's four 4 KB copies
-      mbar_init(&bar->x_empty[i], 4);    // one arrival per warp of the peer's group
+    for (int i = 0; i < 8; ++i) {
+      mbar_init(&bar->x_full[i], 1);     // receiving warp's expect_tx + the peer warp's 4 KB copy
+      mbar_init(&bar->x_empty[i], 1);    // the peer warp has consumed this warp's last copy
     }
     mbar_init(&bar->o_empty, kSoftmaxThreads);
     mbar_init(&bar->sync_all, kSoftmaxThreads);
@@ -179,6 +182,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmKV);
     tma_prefetch_desc(&tmPE);
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmO);
+    tma_prefetch_desc(&tmPart);
   }
   if (warp == 1) tmem_alloc(&bar->tmem_slot, kTmemCols);
   tc_fence_before();
@@ -188,35 +194,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bar->tmem_slot;
 
   PieceIter it;
-  it.init(p.row_prefix, p.rows, e0, e1);
+  it.init(p.row_prefix, p.rows, e0, e1, row0);
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
+    // Ring slot sequence per piece: this CTA's query slabs (the 128 x 64 column blocks of the
+    // absorbed query it owns, 16 KB each), then the piece's cache tiles.
     if (elect_one()) {
       const uint64_t pol = policy_evict_first();
-      int g = 0;
-      int last_tile[kStages];
-      for (int s = 0; s < kStages; ++s) last_tile[s] = -1;
+      // L2 look-ahead: a second cursor over the same tiles, kL2Ahead tiles in front of the ring
+      // loads, has the TMA unit pull its tiles into L2, so the bytes in flight from HBM are not
+      // limited by the ring's depth.  Its first kL2Ahead tiles go out before the wait below.
+      PieceIter pf = it;
+      bool pf_live = false, pf_done = false;
+      int pf_b = 0, pf_key = 0, pf_end = 0;
+      auto prefetch_next = [&]() {
+        while (!pf_done) {
+          if (pf_live && pf_key < pf_end) {
+            for (int i = 0; i < 4; ++i) tma_prefetch_l2_3d(&tmKV, col0 + 64 * i, pf_key, pf_b);
+            if (rank == 1) tma_prefetch_l2_3d(&tmPE, 0, pf_key, pf_b);
+            pf_key += kNK;
+            return;
+          }
+          if (pf_live) pf.next();
+          int r, a, e, n;
+          bool fr;
+          if (!pf.get(r, a, e, n, fr)) {
+            pf_done = true;
+            return;
+          }
+          pf_live = true;
+          pf_b = r / p.T;
+          pf_key = a;
+          pf_end = e;
+        }
+      };
+      for (int i = 0; i < kL2Ahead; ++i) prefetch_next();
+      pdl_wait();   // the queries come from the absorption GEMM
+      int rs = 0;   // ring slot sequence number
+      int last_slot[kStages];
+      for (int s = 0; s < kStages; ++s) last_slot[s] = -1;
       int row, k0, k1, nrow;
       bool first_row;
       bool ok = true;
+      auto take_slot = [&](uint32_t bytes) -> int {   // next ring slot, armed for `bytes`
+        const int s = rs % kStages;
+        if (rs >= kStages && !mbar_wait(&bar->kv_empty[s], ((rs / kStages) - 1) & 1, guard))
+          return -1;
+        mbar_arrive_expect_tx(&bar->kv_full[s], bytes);
+        last_slot[s] = rs++;
+        return s;
+      };
       while (ok && it.get(row, k0, k1, nrow, first_row)) {
         const int b = row / p.T;
         const int ntiles = (k1 - k0 + kNK - 1) / kNK;
-        for (int j = 0; j < ntiles; ++j, ++g) {
-          const int s = g % kStages;
-          if (g >= kStages && !mbar_wait(&bar->kv_empty[s], ((g / kStages) - 1) & 1, guard)) {
-            ok = false;
-            break;
-          }
+        for (int i = 0; i < nslabs && ok; ++i) {
+          const int s = take_slot(kSlabQ);
+          if (s < 0) { ok = false; break; }
+          tma_load_3d(sKV + s * kStageBytes, &tmQ, &bar->kv_full[s], col0 + 64 * i, 0, row);
+        }
+        for (int j = 0; j < ntiles && ok; ++j) {
+          const int s = take_slot(nslabs * kSlabKV);
+          if (s < 0) { ok = false; break; }
           uint64_t* fb = &bar->kv_full[s];
-          mbar_arrive_expect_tx(fb, nslabs * kSlabKV);
           uint8_t* dst = sKV + s * kStageBytes;
           const int key = k0 + j * kNK;
           for (int i = 0; i < 4; ++i)
             tma_load_3d_hint(dst + i * kSlabKV, &tmKV, fb, col0 + 64 * i, key, b, pol);
           if (rank == 1) tma_load_3d_hint(dst + 4 * kSlabKV, &tmPE, fb, 0, key, b, pol);
-          last_tile[s] = g;
+          prefetch_next();
         }
         it.next();
       }
@@ -224,7 +270,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int dummy = 0;
         Guard drain{reinterpret_cast<volatile int*>(&dummy), p.status};
         for (int s = 0; s < kStages; ++s)
-          if (last_tile[s] >= 0) mbar_wait(&bar->kv_full[s], (last_tile[s] / kStages) & 1, drain);
+          if (last_slot[s] >= 0) mbar_wait(&bar->kv_full[s], (last_slot[s] / kStages) & 1, drain);
       }
     }
   } else if (warp == 1) {
@@ -232,13 +278,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (elect_one()) {
       const uint32_t idesc_qk = idesc_bf16(128, kNK, false, false);
       const uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
-      int g = 0, pc = 0;
+      int g = 0, pc = 0, rs = 0;
       int row, k0, k1, nrow;
       bool first_row;
-      // P·V for tile t: A = P in TMEM (aliasing the tile's score buffer), B = the stage's four
-      // latent slabs, MN-major (64 value columns per slab, keys along K).
-      auto issue_pv = [&](int t, bool first) -> bool {
-        const int sb = t % kNS, s = t % kStages;
+      // P·V for tile t (ring slot rt): A = P in TMEM (aliasing the tile's score buffer), B = the
+      // stage's four latent slabs, MN-major (64 value columns per slab, keys along K).
+      auto issue_pv = [&](int t, int rt, bool first) -> bool {
+        const int sb = t % kNS, s = rt % kStages;
         if (!mbar_wait(&bar->p_full[sb], (t / kNS) & 1, guard)) return false;
         if (first && pc > 0 && !mbar_wait(&bar->o_empty, (pc - 1) & 1, guard)) return false;
         tc_fence_after();
@@ -256,11 +302,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = true;
       while (ok && it.get(row, k0, k1, nrow, first_row)) {
         const int ntiles = (k1 - k0 + kNK - 1) / kNK;
-        if (!mbar_wait(&bar->q_full, pc & 1, guard)) break;
-        const int g0 = g;
+        // the piece's query half → TMEM, once the previous piece's score MMAs have read the old one
+        if (pc > 0 && !mbar_wait(&bar->q_empty, (pc - 1) & 1, guard)) break;
+        for (int i = 0; i < nslabs && ok; ++i, ++rs) {
+          const int s = rs % kStages;
+          if (!mbar_wait(&bar->kv_full[s], (rs / kStages) & 1, guard)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t q0 = smem_u32(sKV + s * kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tmem_cp_128x256b(tmem + kTmemQ + i * 32 + kk * 8, smem_desc_sw128(q0 + kk * 32, 16, 1024));
+          umma_commit(&bar->kv_empty[s]);
+        }
+        if (!ok) break;
+        const int g0 = g, rs0 = rs;
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
-          const int s = g % kStages, sb = g % kNS;
-          if (!mbar_wait(&bar->kv_full[s], (g / kStages) & 1, guard)) { ok = false; break; }
+          const int s = (rs0 + j) % kStages, sb = g % kNS;
+          if (!mbar_wait(&bar->kv_full[s], ((rs0 + j) / kStages) & 1, guard)) { ok = false; break; }
           tc_fence_after();
           // scores: S[128 x 32] = Q_half (TMEM) x K_half^T (smem, K-major)
           const uint32_t kv0 = smem_u32(sKV + s * kStageBytes);
@@ -274,12 +332,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           umma_commit(&bar->s_full[g % 6]);
           if (j == ntiles - 1) umma_commit(&bar->q_empty);
-          if (j >= 2 && !issue_pv(g - 2, j - 2 == 0)) { ok = false; break; }
+          if (j >= 2 && !issue_pv(g - 2, rs0 + j - 2, j - 2 == 0)) { ok = false; break; }
         }
         if (!ok) break;
         // the piece's last (up to two) P·V products
-        for (int t = (g - 2 > g0 ? g - 2 : g0); t < g && ok; ++t) ok = issue_pv(t, t == g0);
+        for (int t = (g - 2 > g0 ? g - 2 : g0); t < g && ok; ++t)
+          ok = issue_pv(t, rs0 + (t - g0), t == g0);
         if (!ok) break;
+        rs = rs0 + ntiles;
         ++pc;
         it.next();
       }
@@ -304,9 +364,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     float* lsum_x = sRed + 256;                                                  // [2][128]
     const uint32_t y_warp = smem_u32(sY) + grp * kXSlot + quad * 4096;         // this warp's rows
     const uint32_t x_warp_remote = mapa_shared(smem_u32(sX), peer) + grp * kXSlot + quad * 4096;
-    const uint32_t xfull_remote = mapa_shared(smem_u32(&bar->x_full[grp]), peer);
-    const uint32_t xempty_remote = mapa_shared(smem_u32(&bar->x_empty[grp]), peer);
-    const int nqw = rank == 0 ? 128 : 160;                   // query words (2 x bf16) per row
+    // exchange barriers are per warp: warp (group, quad) trades its 32 head rows with the peer
+    // CTA's warp of the same group and quad only
+    const int xw = grp * 4 + quad;
+    const uint32_t xfull_remote = mapa_shared(smem_u32(&bar->x_full[xw]), peer);
+    const uint32_t xempty_remote = mapa_shared(smem_u32(&bar->x_empty[xw]), peer);
     int g = 0, pc = 0;
     int row, k0, k1, nrow;
     bool first_row;
@@ -316,43 +378,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_arrive(&bar->sync_all);
       return warp_wait(&bar->sync_all, (ph_all++) & 1, guard);
     };
+    pdl_wait();   // outputs may still be read by the kernels before this one
     if (tid < 128) seq[tid] = -1;
     if (!sync_all()) ok = false;
 
     while (ok && it.get(row, k0, k1, nrow, first_row)) {
       const int ntiles = (k1 - k0 + kNK - 1) / kNK;
       const int g0 = g;
-      // this CTA's half of the absorbed query → TMEM (after the previous piece's last score
-      // MMA); the two threads of a row (one per group) split its words, all loads in flight
-      {
-        const int nw = nqw / 2;                              // 64 or 80 words per thread
-        const uint4* src = reinterpret_cast<const uint4*>(
-            p.qabs + (static_cast<size_t>(row) * kHPad + h) * kDk + col0) + grp * (nw / 4);
-        uint32_t w[80];
-#pragma unroll
-        for (int i = 0; i < 20; ++i) {
-          if (i < nw / 4) {
-            const uint4 v = __ldg(src + i);
-            w[4 * i] = v.x;
-            w[4 * i + 1] = v.y;
-            w[4 * i + 2] = v.z;
-            w[4 * i + 3] = v.w;
-          }
-        }
-        if (pc > 0 && !warp_wait(&bar->q_empty, (pc - 1) & 1, guard)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 5; ++c) {
-          if (c < nw / 16) {
-            uint32_t ww[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) ww[i] = w[16 * c + i];
-            tmem_st16_u32(tmem + lane_off + kTmemQ + grp * nw + c * 16, ww);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bar->q_full);
+      // ring slot of the piece's first tile: every piece so far (this one included) put its
+      // query slabs into the ring ahead of its tiles
+      const int rs0 = g0 + nslabs * (pc + 1);
 
       float l_g = 0.f;              // this group's partial row sum ...
       float m_used = -INFINITY;     // ... relative to this maximum
@@ -375,7 +410,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
-          if (k >= 1 && !mbar_wait<true>(&bar->x_empty[grp], (k - 1) & 1, guard)) ok = false;
+          if (k >= 1 && !mbar_wait<true>(&bar->x_empty[xw], (k - 1) & 1, guard)) ok = false;
           if (ok) {
             bulk_copy_to_peer(x_warp_remote, y_warp, 4096, xfull_remote);
             bulk_commit();
@@ -384,8 +419,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         // the peer's half of the same tile
-        if (gtid == 0) mbar_arrive_expect_tx(&bar->x_full[grp], kXSlot);
-        if (!warp_wait<true>(&bar->x_full[grp], k & 1, guard)) { ok = false; break; }
+        if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[xw], kXSlot / 4);
+        if (!warp_wait<true>(&bar->x_full[xw], k & 1, guard)) { ok = false; break; }
 #pragma unroll
         for (int c = 0; c < kNK / 4; ++c) {
           const float4 x =
@@ -481,7 +516,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_st16_u32(tmem + lane_off + kTmemS + (t % kNS) * kNK, pk);
         if (nvalid < kNK) {
           // keys past the piece's end: zero their latent rows so garbage cannot reach P·V
-          uint8_t* st = sKV + (t % kStages) * kStageBytes;
+          uint8_t* st = sKV + ((rs0 + j) % kStages) * kStageBytes;
           const int per_slab = (kNK - nvalid) * 8;
           for (int q = gtid; q < per_slab * 4; q += 128) {
             const int slab = q / per_slab;
@@ -524,43 +559,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float lse = (m_fin + log2f(l_tot)) * 0.69314718055994531f;
       const bool whole = (k0 == 0 && k1 == nrow);
       const int ocol = col0 + grp * 128;
-      if (whole) {
-        bf16* dst = p.o_lat + (static_cast<size_t>(row) * p.n_heads + h) * kC + ocol;
+      const int slot = first_row ? 0 : 1;
+      // The warp's 32 rows x 128 columns of O leave through its 4 KB staging slot, one block of
+      // 32 rows x 128 bytes at a time (bf16: 64 columns, fp32: 32 columns), written in the
+      // 128-byte-swizzle layout (lane = row, 16-byte chunk c at c ^ (row & 7)) and stored by one
+      // TMA tile store per block; the warp does not wait for the global writes.
+      uint8_t* stg = sY + grp * kXSlot + quad * 4096;
+      const int nblk = whole ? 2 : 4;
 #pragma unroll 1
-        for (int c = 0; c < 128 / 32; ++c) {
-          float v[32];
-          tmem_ld32(tmem + lane_off + kTmemO + grp * 128 + c * 32, v);
-          if (h < p.n_heads) {
+      for (int blk = 0; blk < nblk; ++blk) {
+        uint32_t w[32];
+        if (whole) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 a;
-              a.x = pack_bf16x2(v[8 * q] * inv_l, v[8 * q + 1] * inv_l);
-              a.y = pack_bf16x2(v[8 * q + 2] * inv_l, v[8 * q + 3] * inv_l);
-              a.z = pack_bf16x2(v[8 * q + 4] * inv_l, v[8 * q + 5] * inv_l);
-              a.w = pack_bf16x2(v[8 * q + 6] * inv_l, v[8 * q + 7] * inv_l);
-              reinterpret_cast<uint4*>(dst + c * 32)[q] = a;
-            }
+          for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tmem_ld32(tmem + lane_off + kTmemO + grp * 128 + blk * 64 + half * 32, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              w[16 * half + i] = pack_bf16x2(v[2 * i] * inv_l, v[2 * i + 1] * inv_l);
           }
+        } else {
+          float v[32];
+          tmem_ld32(tmem + lane_off + kTmemO + grp * 128 + blk * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i] * inv_l);
         }
+        if (blk == nblk - 1) {   // every TMEM read of O is done: the next piece may overwrite it
+          tc_fence_before();
+          mbar_arrive(&bar->o_empty);
+        }
+        if (lane == 0) bulk_wait_read_all();   // the slot's last copy or store has read it
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+              make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (whole) {
+            if (quad * 32 < p.n_heads) tma_store_3d(&tmO, stg, ocol + blk * 64, quad * 32, row);
+          } else {
+            tma_store_2d(&tmPart, stg, ocol + blk * 32, (pair * 2 + slot) * 128 + quad * 32);
+          }
+          bulk_commit();
+        }
+      }
+      if (whole) {
         if (rank == 0 && grp == 0 && p.lse_out && h < p.n_heads)
           p.lse_out[static_cast<size_t>(row) * p.n_heads + h] = lse;
-      } else {
-        const int slot = first_row ? 0 : 1;
-        float* dst = p.part_o + ((static_cast<size_t>(pair) * 2 + slot) * 128 + h) * kC + ocol;
-#pragma unroll 1
-        for (int c = 0; c < 128 / 32; ++c) {
-          float v[32];
-          tmem_ld32(tmem + lane_off + kTmemO + grp * 128 + c * 32, v);
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(dst + c * 32 + i) =
-                make_float4(v[i] * inv_l, v[i + 1] * inv_l, v[i + 2] * inv_l, v[i + 3] * inv_l);
-        }
-        if (rank == 0 && grp == 0)
-          p.part_lse[(static_cast<size_t>(pair) * 2 + slot) * 128 + h] = lse;
+      } else if (rank == 0 && grp == 0) {
+        p.part_lse[(static_cast<size_t>(pair) * 2 + slot) * 128 + h] = lse;
       }
-      tc_fence_before();
-      mbar_arrive(&bar->o_empty);
       ++pc;
       it.next();
     }
@@ -596,10 +646,35 @@ cudaError_t attention_prepare() {
                               kAttnSmem);
 }
 
-cudaError_t launch_attention(const CUtensorMap& tkv, const CUtensorMap& tpe, const AttnParams& p,
-                             int n_pairs, cudaStream_t s, bool pdl) {
+cudaError_t launch_attention(const AttnMaps& m, const AttnParams& p, int n_pairs, cudaStream_t s,
+                             bool pdl) {
   LaunchCfg lc(dim3(2 * n_pairs), dim3(kThreads), kAttnSmem, s, pdl);
-  return cudaLaunchKernelEx(&lc.cfg, latent_attention_kernel, tkv, tpe, p);
+  return cudaLaunchKernelEx(&lc.cfg, latent_attention_kernel, m.kv, m.pe, m.q, m.o, m.part, p);
+}
+
+bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,
+                         int64_t pe_sb, int64_t pe_st, int batch, int max_seq_len, const void* qabs,
+                         int rows, const void* o_lat, int n_heads, const void* part_o, int pairs) {
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  const uint64_t L = static_cast<uint64_t>(max_seq_len), Bt = static_cast<uint64_t>(batch);
+  const uint64_t R = static_cast<uint64_t>(rows), H = static_cast<uint64_t>(n_heads);
+  const uint32_t box_kv[3] = {64, static_cast<uint32_t>(kNK), 1};
+  const uint64_t d_kv[3] = {kC, L, Bt}, s_kv[2] = {static_cast<uint64_t>(kv_st) * 2,
+                                                   static_cast<uint64_t>(kv_sb) * 2};
+  const uint64_t d_pe[3] = {kDr, L, Bt}, s_pe[2] = {static_cast<uint64_t>(pe_st) * 2,
+                                                    static_cast<uint64_t>(pe_sb) * 2};
+  const uint64_t d_q[3] = {kDk, kHPad, R}, s_q[2] = {kDk * 2, kHPad * kDk * 2};
+  const uint32_t box_q[3] = {64, 128, 1};
+  const uint64_t d_o[3] = {kC, H, R}, s_o[2] = {kC * 2, H * kC * 2};
+  const uint32_t box_o[3] = {64, 32, 1};
+  const uint64_t d_p[2] = {kC, static_cast<uint64_t>(pairs) * 2 * 128}, s_p[1] = {kC * 4};
+  const uint32_t box_p[2] = {32, 32};
+  return encode_tiled(&m->kv, bf, 3, kv, d_kv, s_kv, box_kv, sw) &&
+         encode_tiled(&m->pe, bf, 3, pe, d_pe, s_pe, box_kv, sw) &&
+         encode_tiled(&m->q, bf, 3, qabs, d_q, s_q, box_q, sw) &&
+         encode_tiled(&m->o, bf, 3, o_lat, d_o, s_o, box_o, sw) &&
+         encode_tiled(&m->part, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, part_o, d_p, s_p, box_p, sw);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -57,11 +57,26 @@ __device__ void key_prefix_block(const RmsParams& p) {
     p.row_prefix[r + 1] = acc;
   }
   if (bad) atomicCAS(p.status, kDevOk, kDevBadArg);
+  if (p.pair_row) {
+    __syncthreads();   // the whole prefix is written (and visible to this block)
+    const long long total = p.row_prefix[p.rows];
+    const int pairs = active_pairs(total, p.n_pairs, p.min_keys_per_pair);
+    for (int q = t; q < pairs; q += 128)
+      p.pair_row[q] = row_of_key(p.row_prefix, p.rows, pair_begin(total, pairs, q));
+  }
 }
 
 template <int NCH>
 __global__ void __launch_bounds__(128) rmsnorm_kernel(const RmsParams p) {
-  pdl_launch_dependents();   // the wq_b GEMM may start streaming its weight now
+  // The kernels after this one start early (programmatic dependent launch) and the attention
+  // kernel reads the key prefix before it waits for its predecessors: block 0 therefore writes
+  // the prefix first and makes it visible before any block lets the next kernel start.
+  if (blockIdx.x == 0 && p.row_prefix) {
+    key_prefix_block(p);
+    __threadfence();
+    __syncthreads();
+  }
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 4 + warp;
   if (row < p.rows) {
@@ -119,7 +134,6 @@ __global__ void __launch_bounds__(128) rmsnorm_kernel(const RmsParams p) {
           make_float2(static_cast<float>(cs), static_cast<float>(sn));
     }
   }
-  if (blockIdx.x == 0 && p.row_prefix) key_prefix_block(p);
 }
 
 cudaError_t launch_rmsnorm(const RmsParams& p, cudaStream_t s) {

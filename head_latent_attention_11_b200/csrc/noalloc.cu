@@ -30,7 +30,8 @@ constexpr size_t kOffStatus = 0;
 constexpr size_t kOffPrefix = 256;
 constexpr size_t kOffPartO = kOffPrefix + ((static_cast<size_t>(kNoAllocMaxRows) + 1) * 8 + 255) / 256 * 256;
 constexpr size_t kOffPartLse = kOffPartO + static_cast<size_t>(kNoAllocPairs) * 2 * 128 * kC * 4;
-constexpr size_t kScratchBytes = kOffPartLse + static_cast<size_t>(kNoAllocPairs) * 2 * 128 * 4;
+constexpr size_t kOffPairRow = kOffPartLse + static_cast<size_t>(kNoAllocPairs) * 2 * 128 * 4;
+constexpr size_t kScratchBytes = kOffPairRow + 256;
 
 // ~8.5 MB on every device that loads the library, kept until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
@@ -41,32 +42,6 @@ struct DeviceSetup {
 };
 DeviceSetup g_setup[64];
 std::mutex g_setup_mu;
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-bool cache_map(CUtensorMap* m, const void* base, uint64_t width, uint64_t rows, uint64_t batch,
-               int64_t stride_t, int64_t stride_b) {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
-                                         &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return false;
-    fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  cuuint64_t dims[3] = {width, rows, batch};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(stride_t) * 2, static_cast<cuuint64_t>(stride_b) * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kAttnKeysPerTile), 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -112,10 +87,12 @@ extern "C" mla_status mla_latent_attention_noalloc(
   long long* prefix = reinterpret_cast<long long*>(scratch + kOffPrefix);
   float* part_o = reinterpret_cast<float*>(scratch + kOffPartO);
   float* part_lse = reinterpret_cast<float*>(scratch + kOffPartLse);
+  int* pair_row = reinterpret_cast<int*>(scratch + kOffPairRow);
 
-  CUtensorMap tm_kv, tm_pe;
-  if (!cache_map(&tm_kv, kv_cache, kC, max_seq_len, rows, kv_stride_t, kv_stride_b) ||
-      !cache_map(&tm_pe, pe_cache, kDr, max_seq_len, rows, pe_stride_t, pe_stride_b))
+  const int pairs = attention_pairs() < kNoAllocPairs ? attention_pairs() : kNoAllocPairs;
+  AttnMaps am;
+  if (!make_attention_maps(&am, kv_cache, kv_stride_b, kv_stride_t, pe_cache, pe_stride_b,
+                           pe_stride_t, rows, max_seq_len, q_abs, rows, o_lat, n_heads, part_o, pairs))
     return MLA_ERR_INVALID_ARG;
 
   // the internal status word starts at zero on every call; the prefix and partials are
@@ -128,10 +105,12 @@ extern "C" mla_status mla_latent_attention_noalloc(
   rp.start_pos_dev = start_pos;
   rp.max_seq_len = max_seq_len;
   rp.row_prefix = prefix;
+  rp.pair_row = pair_row;
+  rp.n_pairs = pairs;
+  rp.min_keys_per_pair = 256;
   rp.status = st;
   if (launch_key_prefix(rp, stream) != cudaSuccess) return MLA_ERR_CUDA;
 
-  const int pairs = attention_pairs() < kNoAllocPairs ? attention_pairs() : kNoAllocPairs;
   AttnParams ap{};
   ap.row_prefix = prefix;
   ap.qabs = static_cast<const bf16*>(q_abs);
@@ -146,8 +125,9 @@ extern "C" mla_status mla_latent_attention_noalloc(
   ap.max_seq_len = max_seq_len;
   ap.part_o = part_o;
   ap.part_lse = part_lse;
+  ap.pair_row = pair_row;
   ap.status = st;
-  if (launch_attention(tm_kv, tm_pe, ap, pairs, stream, false) != cudaSuccess) return MLA_ERR_CUDA;
+  if (launch_attention(am, ap, pairs, stream, false) != cudaSuccess) return MLA_ERR_CUDA;
 
   CombineParams cp{};
   cp.row_prefix = prefix;
