@@ -400,7 +400,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         float s[kNK];
         tmem_ld32(tmem + lane_off + kTmemS + (t % kNS) * kNK, s);
-        // hand this warp's 32 rows to the peer: stage locally, one bulk copy per warp
+        // hand this warp's 32 rows to the peer: stage locally, one bulk copy per warp (measured
+        // faster than per-thread st.async stores into the peer's slot)
         if (lane == 0) bulk_wait_read_all();
         __syncwarp();
 #pragma unroll
@@ -443,14 +444,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int i = 0; i < kNK; ++i)
             if (i < nvalid) lg[i] = s[i] * p.scale;
         }
+        // the tile maximum on unscaled scores (the scale is positive: it commutes with max); the
+        // exp2 below applies the scale in its FMA
         float mx[8];
+        const float c2 = p.scale_log2;
 #pragma unroll
-        for (int i = 0; i < kNK; ++i) s[i] = i < nvalid ? s[i] * p.scale_log2 : -INFINITY;
+        for (int i = 0; i < kNK; ++i) s[i] = i < nvalid ? s[i] : -INFINITY;
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx[i] = fmaxf(fmaxf(s[i], s[i + 8]), fmaxf(s[i + 16], s[i + 24]));
 #pragma unroll
         for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
-        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c2;
         // running-max decision for tile t (after the other group decided tile t-1)
         float m_prev = -INFINITY;
         if (j > 0) {
@@ -503,7 +507,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t pk[kNK / 2];
         float e[kNK];
 #pragma unroll
-        for (int i = 0; i < kNK; ++i) e[i] = fast_exp2(s[i] - m_dec);
+        for (int i = 0; i < kNK; ++i) e[i] = fast_exp2(fmaf(s[i], c2, -m_dec));
 #pragma unroll
         for (int i = 0; i < kNK / 2; ++i) pk[i] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
 #pragma unroll
@@ -679,7 +683,7 @@ bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_
 
 // ------------------------------------------------------------------------------------------
 // Combine: rows cut between pairs merge their normalised partials by log-sum-exp weights.
-// One warp per (row, head); lane l owns columns l, l+32, ..., l+480.
+// One warp per (row, head) task; lane l owns columns l, l+32, ..., l+480.
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ int pair_of_key(long long total, int pairs, long long e) {
   int q = static_cast<int>((e * pairs) / total);
@@ -689,48 +693,75 @@ __device__ __forceinline__ int pair_of_key(long long total, int pairs, long long
   return q;
 }
 
-__global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
+// Persistent grid (one block per SM, launched once): each warp walks (row, head) tasks.
+constexpr int kCombineThreads = 512;
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineParams p) {
   pdl_launch_dependents();
   pdl_wait();
-  const int r = blockIdx.x;
-  const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (h >= p.n_heads) return;
+  const int warps = gridDim.x * (kCombineThreads / 32);
   const long long total = p.row_prefix[p.rows];
   const int pairs = active_pairs(total, p.n_pairs, p.min_keys_per_pair);
+  for (int task = blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5);
+       task < p.rows * p.n_heads; task += warps) {
+  const int r = task / p.n_heads, h = task - r * p.n_heads;
   const long long R0 = p.row_prefix[r], R1 = p.row_prefix[r + 1];
   const int plo = pair_of_key(total, pairs, R0), phi = pair_of_key(total, pairs, R1 - 1);
-  if (plo == phi) return;   // written by one pair
-  float mx = -INFINITY;
-  for (int q = plo; q <= phi; ++q) {
-    const int slot = (q == plo && pair_begin(total, pairs, q) < R0) ? 1 : 0;
-    mx = fmaxf(mx, p.part_lse[(static_cast<size_t>(q) * 2 + slot) * 128 + h]);
-  }
-  float wsum = 0.f;
+  if (plo == phi) continue;   // written by one pair
+  // online log-sum-exp merge, four pieces' loads in flight at a time
+  constexpr int kBatch = 4;
+  float mx = -INFINITY, wsum = 0.f;
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  for (int q = plo; q <= phi; ++q) {
-    const int slot = (q == plo && pair_begin(total, pairs, q) < R0) ? 1 : 0;
-    const size_t base = (static_cast<size_t>(q) * 2 + slot) * 128 + h;
-    const float w = exp2f((p.part_lse[base] - mx) * 1.4426950408889634f);
-    wsum += w;
-    const float* src = p.part_o + base * kC;
-    float v[16];
+  for (int q0 = plo; q0 <= phi; q0 += kBatch) {
+    float lse[kBatch], v[kBatch][16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __ldg(src + lane + 32 * i);
+    for (int b = 0; b < kBatch; ++b) {
+      const int q = q0 + b;
+      lse[b] = -INFINITY;
+      if (q <= phi) {
+        const int slot = (q == plo && pair_begin(total, pairs, q) < R0) ? 1 : 0;
+        const size_t base = (static_cast<size_t>(q) * 2 + slot) * 128 + h;
+        lse[b] = __ldg(p.part_lse + base);
+        const float* src = p.part_o + base * kC;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) acc[i] = fmaf(w, v[i], acc[i]);
+        for (int i = 0; i < 16; ++i) v[b][i] = __ldg(src + lane + 32 * i);
+      }
+    }
+    float m_new = mx;
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) m_new = fmaxf(m_new, lse[b]);
+    const float f = mx == -INFINITY ? 0.f : exp2f((mx - m_new) * 1.4426950408889634f);
+    wsum *= f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] *= f;
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      if (q0 + b <= phi) {
+        const float w = exp2f((lse[b] - m_new) * 1.4426950408889634f);
+        wsum += w;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = fmaf(w, v[b][i], acc[i]);
+      }
+    }
+    mx = m_new;
   }
   const float inv = 1.f / wsum;
   bf16* dst = p.o_lat + (static_cast<size_t>(r) * p.n_heads + h) * kC;
 #pragma unroll
   for (int i = 0; i < 16; ++i) dst[lane + 32 * i] = __float2bfloat16_rn(acc[i] * inv);
   if (lane == 0 && p.lse_out) p.lse_out[static_cast<size_t>(r) * p.n_heads + h] = mx + logf(wsum);
+  }
 }
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s, bool pdl) {
-  LaunchCfg lc(dim3(p.rows, (p.n_heads + 3) / 4), dim3(128), 0, s, pdl);
+  const long long tasks = static_cast<long long>(p.rows) * p.n_heads;
+  const long long want = (tasks + kCombineThreads / 32 - 1) / (kCombineThreads / 32);
+  const int cap = 2 * attention_pairs();   // one block per SM (registers allow one)
+  LaunchCfg lc(dim3(static_cast<unsigned>(want < cap ? want : cap)), dim3(kCombineThreads), 0, s,
+               pdl);
   return cudaLaunchKernelEx(&lc.cfg, combine_kernel, p);
 }
 

@@ -31,39 +31,48 @@ __device__ __forceinline__ int row_position(const RmsParams& p, int row, bool* b
 }
 
 __device__ void key_prefix_block(const RmsParams& p) {
-  // 128 threads; thread t owns rows [t*chunk, (t+1)*chunk)
-  __shared__ long long part[128];
-  const int t = threadIdx.x;
+  // 128 threads; thread t owns rows [t*chunk, (t+1)*chunk).  Block-wide scan of the per-thread
+  // key counts (warp shuffles, then the four warp totals), then each thread writes its rows'
+  // prefix and assigns the attention pairs whose first key falls in one of its rows.
+  __shared__ long long warp_total[4];
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
   const int chunk = (p.rows + 127) / 128;
   const int r0 = min(p.rows, t * chunk), r1 = min(p.rows, r0 + chunk);
   long long local = 0;
   bool bad = false;
   for (int r = r0; r < r1; ++r) local += row_position(p, r, &bad) + 1;
-  part[t] = local;
-  __syncthreads();
-  if (t == 0) {
-    long long acc = 0;
-    for (int i = 0; i < 128; ++i) {
-      long long v = part[i];
-      part[i] = acc;
-      acc += v;
-    }
+  long long incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
   }
+  if (lane == 31) warp_total[w] = incl;
   __syncthreads();
-  long long acc = part[t];
+  long long acc = incl - local, total = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const long long v = warp_total[i];
+    if (i < w) acc += v;
+    total += v;
+  }
   if (t == 0) p.row_prefix[0] = 0;
+  // pair q begins at key floor(total * q / pairs): it starts in row r iff that key lies in
+  // [prefix[r], prefix[r+1]), i.e. q in [ceil(prefix[r] * pairs / total), ceil(prefix[r+1] * ...))
+  const int pairs = p.pair_row ? active_pairs(total, p.n_pairs, p.min_keys_per_pair) : 0;
+  auto first_pair_at = [&](long long key) -> long long {
+    return (key * pairs + total - 1) / total;
+  };
   for (int r = r0; r < r1; ++r) {
+    const long long R0 = acc;
     acc += row_position(p, r, &bad) + 1;
     p.row_prefix[r + 1] = acc;
+    if (p.pair_row) {
+      const long long q1 = first_pair_at(acc) < pairs ? first_pair_at(acc) : pairs;
+      for (long long q = first_pair_at(R0); q < q1; ++q) p.pair_row[q] = r;
+    }
   }
   if (bad) atomicCAS(p.status, kDevOk, kDevBadArg);
-  if (p.pair_row) {
-    __syncthreads();   // the whole prefix is written (and visible to this block)
-    const long long total = p.row_prefix[p.rows];
-    const int pairs = active_pairs(total, p.n_pairs, p.min_keys_per_pair);
-    for (int q = t; q < pairs; q += 128)
-      p.pair_row[q] = row_of_key(p.row_prefix, p.rows, pair_begin(total, pairs, q));
-  }
 }
 
 template <int NCH>
