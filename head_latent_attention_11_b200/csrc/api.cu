@@ -125,7 +125,7 @@ Layout layout_of(const mla_config* c) {
   L.q_nope = take(rows * H * kDn * 2);
   L.qabs = take(rows * kHPad * kDk * 2);
   L.o_lat = take(rows * H * kC * 2);
-  L.part_o = take(pairs * 2 * 128 * kC * 4);
+  L.part_o = take(pairs * 2 * 128 * kC * 2);
   L.part_lse = take(pairs * 2 * 128 * 4);
   L.prefix = take((rows + 1) * 8);
   L.pair_row = take(pairs * 4);
@@ -160,7 +160,7 @@ struct mla_ctx {
   bf16* q_nope() const { return reinterpret_cast<bf16*>(ws + L.q_nope); }
   bf16* qabs() const { return reinterpret_cast<bf16*>(ws + L.qabs); }
   bf16* o_lat() const { return reinterpret_cast<bf16*>(ws + L.o_lat); }
-  float* part_o() const { return reinterpret_cast<float*>(ws + L.part_o); }
+  __half* part_o() const { return reinterpret_cast<__half*>(ws + L.part_o); }
   float* part_lse() const { return reinterpret_cast<float*>(ws + L.part_lse); }
   long long* prefix() const { return reinterpret_cast<long long*>(ws + L.prefix); }
   int* pair_row() const { return reinterpret_cast<int*>(ws + L.pair_row); }

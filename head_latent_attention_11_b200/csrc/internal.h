@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -88,7 +89,7 @@ struct AttnParams {
   float* lse_out;               // [rows, H] or null
   float* logits;                // [B, H, max_seq_len] or null (decode debug)
   int max_seq_len;
-  float* part_o;                // [pairs, 2, 128, 512] fp32 normalised partial outputs
+  __half* part_o;               // [pairs, 2, 128, 512] fp16 normalised partial outputs
   float* part_lse;              // [pairs, 2, 128]
   const int* pair_row;          // [pairs] first row of each pair's key range, or null
   int* status;
@@ -100,7 +101,7 @@ struct CombineParams {
   int n_heads;
   int n_pairs;                  // pairs the attention kernel launched
   int min_keys_per_pair;
-  const float* part_o;
+  const __half* part_o;
   const float* part_lse;
   bf16* o_lat;
   float* lse_out;
@@ -142,7 +143,7 @@ struct AttnMaps {
   CUtensorMap pe;    // rotary cache  bf16 {64, max_seq_len, batch},  box {64, 32, 1}
   CUtensorMap q;     // absorbed queries bf16 {576, 128, rows},       box {64, 128, 1}
   CUtensorMap o;     // o_lat         bf16 {512, n_heads, rows},      box {64, 32, 1}
-  CUtensorMap part;  // split partials fp32 {512, pairs * 2 * 128},   box {32, 32}
+  CUtensorMap part;  // split partials fp16 {512, pairs * 2 * 128},   box {64, 32}
 };
 // Strides in elements; false if a map cannot be encoded (alignment, sizes).
 bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,

@@ -15,31 +15,35 @@
 //     score tile over them and hands it to the peer; both CTAs then hold identical full scores
 //     and run the identical online softmax.  Each CTA accumulates the value half it owns,
 //     O[128 x 256] fp32 in TMEM.
-//   * The CTA's half of the absorbed query lives in TMEM and is the A operand of the score MMA;
-//     the probabilities P (bf16) overwrite the score tile in TMEM and are the A operand of the
-//     P·V MMA.  Shared memory holds the cache ring (32-key tiles, 7 stages, TMA with 128-byte
-//     swizzle, evict-first) and the exchange buffers.
-//     TMEM columns: O [0,256) | query half [256,416) | three 32-column score/P buffers [416,512).
-//     With three buffers the score MMA of tile g only waits for P·V of tile g-3, so the tensor
-//     core runs two tiles ahead of the softmax.
-//   * Score exchange: partial tiles go through a local staging buffer to the bulk-copy engine
-//     (shared::cta → the peer's shared memory), which completes a transaction count on the
-//     peer's barrier.
-//   * Eight softmax warps in two groups of four that take alternate tiles (ping-pong); within a
-//     group one thread owns one head row.  Only the running-max decision is handed from tile to
-//     tile across the groups (per-row flag in shared memory); each group keeps its own partial
-//     row sum, so the softmax work of consecutive tiles overlaps.
-//   * Each warp stages its 32 rows of partial scores and ships them with its own 4 KB bulk copy;
-//     it waits only for the copy of its counterpart warp (same group and lane quarter) in the
-//     peer CTA, through a barrier pair of its own.
+//   * The CTA's 256 latent query columns live in TMEM (A operand of the score MMA); rank 1's 64
+//     rotary query columns stay in shared memory (A from a smem descriptor for those K-steps), so
+//     both CTAs have room for four score buffers.  The query reaches TMEM by TMA into ring slots
+//     and tcgen05.cp, once per piece.  The probabilities P (bf16) overwrite the score tile in
+//     TMEM and are the A operand of P·V.  Shared memory holds the cache ring (32-key tiles, 7
+//     stages, TMA with 128-byte swizzle, evict-first) and the exchange buffers.
+//     TMEM columns: O [0,256) | latent query [256,384) | four 32-column score/P buffers [384,512).
+//     With four buffers the score MMA of tile g only waits for P·V of tile g-4 to be issued.
+//   * Score exchange: each warp stages its 32 rows of partial scores and ships them with one
+//     4 KB bulk copy (shared::cta → the peer's receive slot), which completes a transaction count
+//     on the peer warp's own barrier; a warp waits only for its counterpart (same group and lane
+//     quarter) in the peer CTA.  The four warps of a lane quarter share one staging slot, handed
+//     from use to use in a fixed order.
+//   * Twelve softmax warps in three groups of four take turns by tile; within a group one thread
+//     owns one head row.  Only the running-max decision is handed from tile to tile across the
+//     groups (per-row flag in shared memory); each group keeps its own partial row sum, so the
+//     softmax work of consecutive tiles overlaps.
 //   * The flattened key range of all rows is split evenly over the cluster pairs (split-K over
 //     keys, also across row boundaries); a row cut between pairs leaves normalised partials
-//     (O/l, lse) for the combine kernel, an uncut row is written as bf16 o_lat directly.
+//     (O/l, lse) for the combine kernel, an uncut row is written as bf16 o_lat directly, both
+//     by TMA tile stores from a swizzled staging block.
 //   * Online softmax in exp2 domain with lazy rescaling: the running max is only raised (and O
 //     in TMEM rescaled) when a tile's max exceeds it by more than 8 (factor 256), which keeps the
 //     rescale off the common path while the result stays exact.
-//   * Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-9 query loader,
-//     softmax and epilogue (thread pair = head row = TMEM lane).
+//   * Warp roles: warp 0 TMA producer (lane 1 of rank 1: rotary query slab), warp 1 TMEM owner
+//     + score-MMA issuer (and the query copies), warp 2 P·V issuer, warps 3-14 softmax and
+//     epilogue (thread = head row = TMEM lane).  A tcgen05 instruction costs a single issuing
+//     thread ~48 cycles, so the score and P·V streams are issued by two threads in parallel.
+//     The score buffer a QK reuses is handed back by the P·V thread's completion barrier.
 //   * Every wait is bounded (see tc100.cuh); a stuck pipeline records a status and ends.
 #include "internal.h"
 #include "tc100.cuh"
@@ -55,38 +59,46 @@ constexpr int kSlabKV = kNK * 128;         // 4 KB: 64 columns x 32 keys, bf16
 constexpr int kMaxSlabs = 5;               // rank 1: 4 latent slabs + 1 rotary slab
 constexpr int kSlabQ = 128 * 64 * 2;       // 16 KB: 64 query columns of all 128 head rows
 constexpr int kStageBytes = kMaxSlabs * kSlabKV;
-constexpr int kXSlot = 128 * kNK * 4;      // 16 KB: one partial score tile, fp32
+constexpr int kGroups = 3;                 // softmax groups (4 warps each) taking turns by tile
+constexpr int kXWarp = 32 * kNK * 4;       // 4 KB: one warp's 32 rows of a partial score tile
 
 constexpr int kOffKV = 0;
-constexpr int kOffX = kOffKV + kStages * kStageBytes;     // receive slots (peer → this CTA)
-constexpr int kOffY = kOffX + 2 * kXSlot;                 // staging slots (this CTA → peer)
-constexpr int kOffRed = kOffY + 2 * kXSlot;               // row-max / row-sum exchange
-constexpr int kOffBar = kOffRed + 3 * 2 * 128 * 4;
-constexpr int kAttnSmem = kOffBar + 512 + 1024;
+constexpr int kOffX = kOffKV + kStages * kStageBytes;     // receive slots (peer → this CTA), per warp
+constexpr int kOffY = kOffX + kGroups * 4 * kXWarp;       // staging slots, one per lane quarter
+constexpr int kOffQPe = kOffY + 4 * kXWarp;               // rank 1: rotary query slab (A from smem)
+constexpr int kOffRed = kOffQPe + kSlabQ;                 // row-max / row-sum exchange
+constexpr int kOffBar = kOffRed + (2 + 2 * kGroups) * 128 * 4;
+constexpr int kAttnSmem = kOffBar + 768 + 1024;
 
 constexpr int kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;             // [0, 256)
-constexpr uint32_t kTmemQ = 256;           // [256, 416): up to 320 bf16 K-columns
-constexpr uint32_t kTmemS = 416;           // three 32-column score / probability buffers
-constexpr int kNS = 3;
+constexpr uint32_t kTmemQ = 256;           // [256, 384): 256 bf16 latent query columns
+constexpr uint32_t kTmemS = 384;           // four 32-column score / probability buffers
+constexpr int kNS = 4;
+constexpr int kNB = 8;                     // ring of per-tile barrier slots (s_full, pv_done)
 
-constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxWarps = 4 * kGroups;
 constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
-constexpr int kThreads = 64 + kSoftmaxThreads;
+constexpr int kThreads = 96 + kSoftmaxThreads;
+constexpr int kSoftmaxWarp0 = 3;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t q_empty;         // the piece's last score MMA has read the query in TMEM
-  uint64_t s_full[6], p_full[kNS], pv_done[6];
+  uint64_t q_empty;         // the piece's last score MMA has read the query (TMEM and smem)
+  uint64_t qpe_full;        // rank 1: the piece's rotary query slab has landed
+  uint64_t s_full[kNB], p_full[kNS], pv_done[kNB];
   uint64_t o_empty;
-  uint64_t x_full[8], x_empty[8];   // [group][warp quad]
-  uint64_t sync_all;       // the 256 softmax threads
+  uint64_t x_full[4 * kGroups], x_empty[4 * kGroups];   // [group][warp quad]
+  uint64_t sync_all;        // all softmax threads
   uint64_t drain;
   uint32_t tmem_slot;
   int abort_flag;
+  // staging slot of each lane quarter: number of uses that have released it (a counter, not a
+  // barrier: a warp may start waiting for its turn more than one use ahead)
+  int y_released[4];
 };
-static_assert(sizeof(Bars) <= 512, "barrier block");
+static_assert(sizeof(Bars) <= 768, "barrier block");
 static_assert(kAttnSmem <= 232448, "shared memory budget");
 
 // Iterates the pieces (row, [k0, k1)) of one pair's key range.
@@ -117,10 +129,6 @@ struct PieceIter {
   __device__ void next() { ++r; }
 };
 
-__device__ __forceinline__ uint32_t xbuf_off(int slot, int h, int c) {
-  // row h of a slot holds 32 floats = 8 chunks of 16 B; chunk c is stored at (c + h) & 7
-  return static_cast<uint32_t>(slot * kXSlot + h * 128 + (((c + h) & 7) << 4));
-}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     latent_attention_kernel(const __grid_constant__ CUtensorMap tmKV,
@@ -156,8 +164,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const long long e0 = pair_begin(total, pairs, pair), e1 = pair_begin(total, pairs, pair + 1);
 
   const int warp = static_cast<int>(warp_id());
-  const int nslabs = rank == 0 ? 4 : 5;           // 64-column slabs this CTA owns
+  const int nslabs = rank == 0 ? 4 : 5;           // 64-column cache slabs this CTA owns
   const int col0 = rank == 0 ? 0 : 256;           // first cache / query column it owns
+  uint8_t* sQPe = smem + kOffQPe;                 // rank 1: the rotary query slab
   Guard guard{reinterpret_cast<volatile int*>(&bar->abort_flag), p.status};
 
   if (threadIdx.x == 0) {
@@ -166,18 +175,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&bar->kv_empty[i], 1);
     }
     mbar_init(&bar->q_empty, 1);
-    for (int i = 0; i < 6; ++i) {
+    mbar_init(&bar->qpe_full, 1);
+    for (int i = 0; i < kNB; ++i) {
       mbar_init(&bar->s_full[i], 1);
       mbar_init(&bar->pv_done[i], 1);
     }
     for (int i = 0; i < kNS; ++i) mbar_init(&bar->p_full[i], 128);   // the tile's group
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 4 * kGroups; ++i) {
       mbar_init(&bar->x_full[i], 1);     // receiving warp's expect_tx + the peer warp's 4 KB copy
       mbar_init(&bar->x_empty[i], 1);    // the peer warp has consumed this warp's last copy
     }
+    for (int i = 0; i < 4; ++i) bar->y_released[i] = 0;
     mbar_init(&bar->o_empty, kSoftmaxThreads);
     mbar_init(&bar->sync_all, kSoftmaxThreads);
-    mbar_init(&bar->drain, 1);
+    mbar_init(&bar->drain, 2);   // both MMA-issuing threads
     bar->abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmKV);
@@ -198,9 +209,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    // Ring slot sequence per piece: this CTA's query slabs (the 128 x 64 column blocks of the
-    // absorbed query it owns, 16 KB each), then the piece's cache tiles.
-    if (elect_one()) {
+    // Lane 0: ring slot sequence per piece = the 4 latent query slabs this CTA owns (128 x 64
+    // columns, 16 KB each), then the piece's cache tiles.  Lane 1 of rank 1: the piece's rotary
+    // query slab into its own buffer, once the previous piece's last score MMA has read it.
+    const uint32_t lane = lane_id();
+    if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       // L2 look-ahead: a second cursor over the same tiles, kL2Ahead tiles in front of the ring
       // loads, has the TMA unit pull its tiles into L2, so the bytes in flight from HBM are not
@@ -248,7 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       while (ok && it.get(row, k0, k1, nrow, first_row)) {
         const int b = row / p.T;
         const int ntiles = (k1 - k0 + kNK - 1) / kNK;
-        for (int i = 0; i < nslabs && ok; ++i) {
+        for (int i = 0; i < 4 && ok; ++i) {
           const int s = take_slot(kSlabQ);
           if (s < 0) { ok = false; break; }
           tma_load_3d(sKV + s * kStageBytes, &tmQ, &bar->kv_full[s], col0 + 64 * i, 0, row);
@@ -272,39 +285,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s)
           if (last_slot[s] >= 0) mbar_wait(&bar->kv_full[s], (last_slot[s] / kStages) & 1, drain);
       }
+    } else if (lane == 1 && rank == 1) {
+      pdl_wait();
+      int row, k0, k1, nrow, pc = 0;
+      bool first_row;
+      bool armed = false;
+      while (it.get(row, k0, k1, nrow, first_row)) {
+        if (pc > 0 && !mbar_wait(&bar->q_empty, (pc - 1) & 1, guard)) break;
+        mbar_arrive_expect_tx(&bar->qpe_full, kSlabQ);
+        armed = true;
+        tma_load_3d(sQPe, &tmQ, &bar->qpe_full, kC, 0, row);
+        ++pc;
+        it.next();
+      }
+      if (armed && guard.aborted()) {
+        int dummy = 0;
+        Guard drain{reinterpret_cast<volatile int*>(&dummy), p.status};
+        mbar_wait(&bar->qpe_full, (pc - 1) & 1, drain);
+      }
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
+    // ---------------------------------------------------------------- score-MMA issuer
     if (elect_one()) {
       const uint32_t idesc_qk = idesc_bf16(128, kNK, false, false);
-      const uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
       int g = 0, pc = 0, rs = 0;
       int row, k0, k1, nrow;
       bool first_row;
-      // P·V for tile t (ring slot rt): A = P in TMEM (aliasing the tile's score buffer), B = the
-      // stage's four latent slabs, MN-major (64 value columns per slab, keys along K).
-      auto issue_pv = [&](int t, int rt, bool first) -> bool {
-        const int sb = t % kNS, s = rt % kStages;
-        if (!mbar_wait(&bar->p_full[sb], (t / kNS) & 1, guard)) return false;
-        if (first && pc > 0 && !mbar_wait(&bar->o_empty, (pc - 1) & 1, guard)) return false;
-        tc_fence_after();
-        const uint32_t b0 = smem_u32(sKV + s * kStageBytes);
-#pragma unroll
-        for (int k = 0; k < kNK / 16; ++k) {
-          umma_bf16_tmem_a(tmem + kTmemO, tmem + kTmemS + sb * kNK + k * 8,
-                           smem_desc_sw128(b0 + k * 2048, kSlabKV, 1024), idesc_pv,
-                           (first && k == 0) ? 0u : 1u);
-        }
-        umma_commit(&bar->kv_empty[s]);
-        umma_commit(&bar->pv_done[t % 6]);
-        return true;
-      };
+      const uint32_t qpe0 = smem_u32(sQPe);
       bool ok = true;
       while (ok && it.get(row, k0, k1, nrow, first_row)) {
         const int ntiles = (k1 - k0 + kNK - 1) / kNK;
-        // the piece's query half → TMEM, once the previous piece's score MMAs have read the old one
+        // the piece's latent query half → TMEM, once the previous piece's score MMAs have read the
+        // old one (its rotary slab is reloaded by the producer after the same point)
         if (pc > 0 && !mbar_wait(&bar->q_empty, (pc - 1) & 1, guard)) break;
-        for (int i = 0; i < nslabs && ok; ++i, ++rs) {
+        for (int i = 0; i < 4 && ok; ++i, ++rs) {
           const int s = rs % kStages;
           if (!mbar_wait(&bar->kv_full[s], (rs / kStages) & 1, guard)) { ok = false; break; }
           tc_fence_after();
@@ -315,14 +329,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           umma_commit(&bar->kv_empty[s]);
         }
         if (!ok) break;
-        const int g0 = g, rs0 = rs;
+        if (rank == 1 && !mbar_wait(&bar->qpe_full, pc & 1, guard)) break;
+        const int rs0 = rs;
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
           const int s = (rs0 + j) % kStages, sb = g % kNS;
           if (!mbar_wait(&bar->kv_full[s], ((rs0 + j) / kStages) & 1, guard)) { ok = false; break; }
+          // the score buffer held P of tile g - kNS: its P·V (other thread) must have completed
+          if (g >= kNS && !mbar_wait(&bar->pv_done[(g - kNS) % kNB], ((g - kNS) / kNB) & 1, guard)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          // scores: S[128 x 32] = Q_half (TMEM) x K_half^T (smem, K-major)
+          // scores: S[128 x 32] = Q_half x K_half^T: latent part with the query in TMEM, the
+          // rotary part (rank 1) with the query slab in shared memory; cache K-major in smem
           const uint32_t kv0 = smem_u32(sKV + s * kStageBytes);
-          for (int i = 0; i < nslabs; ++i) {
+          for (int i = 0; i < 4; ++i) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               umma_bf16_tmem_a(tmem + kTmemS + sb * kNK, tmem + kTmemQ + i * 32 + kk * 8,
@@ -330,14 +351,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                (i | kk) != 0);
             }
           }
-          umma_commit(&bar->s_full[g % 6]);
+          if (rank == 1) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              umma_bf16(tmem + kTmemS + sb * kNK, smem_desc_sw128(qpe0 + kk * 32, 16, 1024),
+                        smem_desc_sw128(kv0 + 4 * kSlabKV + kk * 32, 16, 1024), idesc_qk, 1u);
+            }
+          }
+          umma_commit(&bar->s_full[g % kNB]);
           if (j == ntiles - 1) umma_commit(&bar->q_empty);
-          if (j >= 2 && !issue_pv(g - 2, rs0 + j - 2, j - 2 == 0)) { ok = false; break; }
         }
-        if (!ok) break;
-        // the piece's last (up to two) P·V products
-        for (int t = (g - 2 > g0 ? g - 2 : g0); t < g && ok; ++t)
-          ok = issue_pv(t, rs0 + (t - g0), t == g0);
         if (!ok) break;
         rs = rs0 + ntiles;
         ++pc;
@@ -345,31 +368,100 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       umma_commit(&bar->drain);
     }
+  } else if (warp == 2) {
+    // ---------------------------------------------------------------- P·V issuer
+    // P·V for tile t: A = P in TMEM (aliasing the tile's score buffer), B = the ring stage's four
+    // latent slabs, MN-major (64 value columns per slab, keys along K).  P is complete (p_full)
+    // only after the score MMA of the tile has finished reading the stage.
+    if (elect_one()) {
+      const uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
+      int g = 0, pc = 0;
+      int row, k0, k1, nrow;
+      bool first_row;
+      bool ok = true;
+      while (ok && it.get(row, k0, k1, nrow, first_row)) {
+        const int ntiles = (k1 - k0 + kNK - 1) / kNK;
+        const int rs0 = g + 4 * (pc + 1);   // ring slot of the piece's first tile
+        for (int j = 0; j < ntiles && ok; ++j, ++g) {
+          const int sb = g % kNS, s = (rs0 + j) % kStages;
+          if (!mbar_wait(&bar->p_full[sb], (g / kNS) & 1, guard)) { ok = false; break; }
+          if (j == 0 && pc > 0 && !mbar_wait(&bar->o_empty, (pc - 1) & 1, guard)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b0 = smem_u32(sKV + s * kStageBytes);
+#pragma unroll
+          for (int k = 0; k < kNK / 16; ++k) {
+            umma_bf16_tmem_a(tmem + kTmemO, tmem + kTmemS + sb * kNK + k * 8,
+                             smem_desc_sw128(b0 + k * 2048, kSlabKV, 1024), idesc_pv,
+                             (j == 0 && k == 0) ? 0u : 1u);
+          }
+          umma_commit(&bar->kv_empty[s]);
+          umma_commit(&bar->pv_done[g % kNB]);
+        }
+        if (!ok) break;
+        ++pc;
+        it.next();
+      }
+      umma_commit(&bar->drain);
+    }
   } else {
-    // ---------------------------------------------------------------- query load, softmax, epilogue
-    // Two groups of four warps take alternate tiles (group = global tile index & 1); within a
-    // group a thread owns one head row (TMEM lane) and all 32 keys of its tiles.  The running
-    // maximum of a row is handed from tile to tile across the groups through m_ref / seq in
-    // shared memory; each group keeps its own partial row sum relative to the last maximum it
-    // used, so the two groups' softmax work overlaps and only the max decision is sequential.
+    // ---------------------------------------------------------------- softmax, epilogue
+    // kGroups groups of four warps take turns by tile (group = global tile index % kGroups);
+    // within a group a thread owns one head row (TMEM lane) and all 32 keys of its tiles.  The
+    // running maximum of a row is handed from tile to tile across the groups through m_ref / seq
+    // in shared memory; each group keeps its own partial row sum relative to the last maximum it
+    // used, so the groups' softmax work overlaps and only the max decision is sequential.
+    //
+    // Staging: the four warps of a lane quarter (one per group) share one 4 KB slot for their
+    // outgoing score copies and for the epilogue's TMA stores.  Uses of a slot are numbered in a
+    // fixed order (the pieces' tiles, then each piece's epilogue blocks, group 0 before group 1)
+    // and handed on through a release counter: use u waits until u uses have released it.
     const int quad = warp & 3;
-    const int grp = (warp - 2) >> 2;                         // 0: warps 2-5, 1: warps 6-9
+    const int grp = (warp - kSoftmaxWarp0) >> 2;             // warps 3-6, 7-10, 11-14
     const int lane = static_cast<int>(lane_id());
     const int h = quad * 32 + lane;                          // head row = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const int tid = static_cast<int>(threadIdx.x) - 64;      // 0..255
+    const int tid = static_cast<int>(threadIdx.x) - 32 * kSoftmaxWarp0;   // 0..kSoftmaxThreads-1
     const int gtid = tid & 127;                              // thread index within the group
     volatile float* m_ref = reinterpret_cast<volatile float*>(sRed);            // [128]
     volatile int* seq = reinterpret_cast<volatile int*>(sRed + 128);            // [128]
-    float* lsum_x = sRed + 256;                                                  // [2][128]
-    const uint32_t y_warp = smem_u32(sY) + grp * kXSlot + quad * 4096;         // this warp's rows
-    const uint32_t x_warp_remote = mapa_shared(smem_u32(sX), peer) + grp * kXSlot + quad * 4096;
-    // exchange barriers are per warp: warp (group, quad) trades its 32 head rows with the peer
-    // CTA's warp of the same group and quad only
-    const int xw = grp * 4 + quad;
+    float* lsum_x = sRed + 256;                       // [piece parity][kGroups][128]
+    uint8_t* stg = sY + quad * kXWarp;                       // this lane quarter's staging slot
+    const int xw = grp * 4 + quad;                           // this warp's receive slot / barriers
+    uint8_t* xslot = sX + xw * kXWarp;
+    const uint32_t x_remote = mapa_shared(smem_u32(xslot), peer);
     const uint32_t xfull_remote = mapa_shared(smem_u32(&bar->x_full[xw]), peer);
     const uint32_t xempty_remote = mapa_shared(smem_u32(&bar->x_empty[xw]), peer);
-    int g = 0, pc = 0;
+    // row r of a warp's 4 KB score block: 32 floats = 8 chunks of 16 B, chunk c at (c + r) & 7
+    auto xoff = [](int r, int c) -> int { return r * 128 + (((c + r) & 7) << 4); };
+    volatile int* y_released = bar->y_released + quad;
+    auto acquire_stage = [&](int u) -> bool {   // wait until uses 0..u-1 released the slot
+      bool got = true;
+      if (*y_released < u) {
+        const unsigned long long t0 = globaltimer_ns();
+        uint32_t n = 0;
+        while (*y_released < u) {
+          if ((++n & 63u) == 0 && (guard.aborted() || globaltimer_ns() - t0 > kWaitLimitNs)) {
+            if (!guard.aborted()) guard.fail(kDevTimeout);
+            got = false;
+            break;
+          }
+        }
+      }
+      got = __all_sync(0xffffffffu, got);
+      __threadfence_block();
+      return got;
+    };
+    auto release_stage = [&](int u) {           // the slot's copy / store has read it: hand on
+      if (lane == 0) {
+        bulk_wait_read_all();
+        __threadfence_block();
+        *y_released = u + 1;
+      }
+    };
+    int g = 0, pc = 0, ubase = 0;   // tiles before this piece, pieces, extra slot uses before
     int row, k0, k1, nrow;
     bool first_row;
     bool ok = true;
@@ -386,46 +478,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int ntiles = (k1 - k0 + kNK - 1) / kNK;
       const int g0 = g;
       // ring slot of the piece's first tile: every piece so far (this one included) put its
-      // query slabs into the ring ahead of its tiles
-      const int rs0 = g0 + nslabs * (pc + 1);
+      // four query slabs into the ring ahead of its tiles
+      const int rs0 = g0 + 4 * (pc + 1);
+      const bool whole = (k0 == 0 && k1 == nrow);
+      constexpr int nblk = 2;           // epilogue blocks of 64 columns per writing group
+      // group 1 stages its epilogue in its own receive slot when it had a tile in this piece (the
+      // peer may refill that slot only after the epilogue: its last release is held back);
+      // otherwise it queues on the lane quarter's shared slot behind group 0
+      const bool g1_has_tile = ((1 - g0 % kGroups + kGroups) % kGroups) < ntiles;
+      bool xe_held = false;
 
       float l_g = 0.f;              // this group's partial row sum ...
       float m_used = -INFINITY;     // ... relative to this maximum
-      int j = ((g0 & 1) == grp) ? 0 : 1;
-      for (; j < ntiles; j += 2) {
+      int j = ((grp - g0 % kGroups) + kGroups) % kGroups;
+      for (; j < ntiles; j += kGroups) {
         const int t = g0 + j;
-        const int k = t >> 1;       // per-group tile counter (exchange slot phases)
+        const int k = t / kGroups;  // per-group tile counter (exchange slot phases)
         // scores of this CTA's columns
-        if (!warp_wait(&bar->s_full[t % 6], (t / 6) & 1, guard)) { ok = false; break; }
+        if (!warp_wait(&bar->s_full[t % kNB], (t / kNB) & 1, guard)) { ok = false; break; }
         tc_fence_after();
         float s[kNK];
         tmem_ld32(tmem + lane_off + kTmemS + (t % kNS) * kNK, s);
-        // hand this warp's 32 rows to the peer: stage locally, one bulk copy per warp (measured
-        // faster than per-thread st.async stores into the peer's slot)
-        if (lane == 0) bulk_wait_read_all();
-        __syncwarp();
+        // hand this warp's 32 rows to the peer: stage locally, one 4 KB bulk copy per warp
+        if (!acquire_stage(t + ubase)) { ok = false; break; }
 #pragma unroll
         for (int c = 0; c < kNK / 4; ++c)
-          *reinterpret_cast<float4*>(sY + grp * kXSlot + xbuf_off(0, h, c)) =
+          *reinterpret_cast<float4*>(stg + xoff(lane, c)) =
               make_float4(s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
           if (k >= 1 && !mbar_wait<true>(&bar->x_empty[xw], (k - 1) & 1, guard)) ok = false;
           if (ok) {
-            bulk_copy_to_peer(x_warp_remote, y_warp, 4096, xfull_remote);
+            bulk_copy_to_peer(x_remote, smem_u32(stg), kXWarp, xfull_remote);
             bulk_commit();
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
+        release_stage(t + ubase);   // as soon as the copy has read the slot
         // the peer's half of the same tile
-        if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[xw], kXSlot / 4);
+        if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[xw], kXWarp);
         if (!warp_wait<true>(&bar->x_full[xw], k & 1, guard)) { ok = false; break; }
 #pragma unroll
         for (int c = 0; c < kNK / 4; ++c) {
-          const float4 x =
-              *reinterpret_cast<const float4*>(sX + grp * kXSlot + xbuf_off(0, h, c));
+          const float4 x = *reinterpret_cast<const float4*>(xslot + xoff(lane, c));
           s[4 * c] += x.x;
           s[4 * c + 1] += x.y;
           s[4 * c + 2] += x.z;
@@ -434,7 +531,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // every lane has consumed its loads from the slot before lane 0 lets the peer refill it
         consume32(s);
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote_relaxed(xempty_remote);
+        if (grp == 1 && j + kGroups >= ntiles) xe_held = true;   // released after the epilogue
+        else if (lane == 0) mbar_arrive_remote_relaxed(xempty_remote);
         const int key0 = k0 + j * kNK;
         const int nvalid = min(kNK, k1 - key0);
         if (p.logits && rank == 0 && h < p.n_heads) {
@@ -455,7 +553,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
         const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c2;
-        // running-max decision for tile t (after the other group decided tile t-1)
+        // running-max decision for tile t (after another group decided tile t-1)
         float m_prev = -INFINITY;
         if (j > 0) {
           bool seen = true;
@@ -481,7 +579,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // O holds tiles up to t-1: if any row of the warp raises its maximum, the warp waits for
         // their last P·V and rescales (factor 1 for the other rows) — warp-uniform TMEM access
         if (j > 0 && __any_sync(0xffffffffu, raise)) {
-          if (!warp_wait(&bar->pv_done[(t - 1) % 6], ((t - 1) / 6) & 1, guard)) { ok = false; break; }
+          if (!warp_wait(&bar->pv_done[(t - 1) % kNB], ((t - 1) / kNB) & 1, guard)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const float f = raise ? fast_exp2(m_prev - m_new) : 1.f;
 #pragma unroll 1
@@ -505,18 +606,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         // probabilities → TMEM (over the score buffer), row sum
         uint32_t pk[kNK / 2];
-        float e[kNK];
 #pragma unroll
-        for (int i = 0; i < kNK; ++i) e[i] = fast_exp2(fmaf(s[i], c2, -m_dec));
+        for (int i = 0; i < kNK; ++i) s[i] = fast_exp2(fmaf(s[i], c2, -m_dec));
 #pragma unroll
-        for (int i = 0; i < kNK / 2; ++i) pk[i] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
+        for (int i = 0; i < kNK / 2; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) e[i] += e[i + 16];
+        for (int i = 0; i < 16; ++i) s[i] += s[i + 16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) e[i] += e[i + 8];
+        for (int i = 0; i < 8; ++i) s[i] += s[i + 8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) e[i] += e[i + 4];
-        l_g += (e[0] + e[2]) + (e[1] + e[3]);
+        for (int i = 0; i < 4; ++i) s[i] += s[i + 4];
+        l_g += (s[0] + s[2]) + (s[1] + s[3]);
         tmem_st16_u32(tmem + lane_off + kTmemS + (t % kNS) * kNK, pk);
         if (nvalid < kNK) {
           // keys past the piece's end: zero their latent rows so garbage cannot reach P·V
@@ -538,7 +638,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
       // ------------------------------------------------------------ epilogue of the piece
       const int glast = g - 1;
-      // final maximum of the row (decided at the last tile), both groups' sums relative to it
+      // final maximum of the row (decided at the last tile), all groups' sums relative to it
       {
         bool seen = true;
         const unsigned long long t0 = globaltimer_ns();
@@ -554,60 +654,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       __threadfence_block();
       const float m_fin = m_ref[h];
-      lsum_x[grp * 128 + h] = (m_used == -INFINITY) ? 0.f : l_g * fast_exp2(m_used - m_fin);
+      // (double-buffered by piece: a group cannot pass the next piece's sync_all before every
+      // group has read this piece's sums)
+      float* lsum = lsum_x + (pc & 1) * kGroups * 128;
+      lsum[grp * 128 + h] = (m_used == -INFINITY) ? 0.f : l_g * fast_exp2(m_used - m_fin);
       if (!sync_all()) break;
-      const float l_tot = lsum_x[h] + lsum_x[128 + h];
-      if (!warp_wait(&bar->pv_done[glast % 6], (glast / 6) & 1, guard)) break;
-      tc_fence_after();
+      float l_tot = 0.f;
+#pragma unroll
+      for (int G = 0; G < kGroups; ++G) l_tot += lsum[G * 128 + h];
       const float inv_l = 1.f / l_tot;
       const float lse = (m_fin + log2f(l_tot)) * 0.69314718055994531f;
-      const bool whole = (k0 == 0 && k1 == nrow);
-      const int ocol = col0 + grp * 128;
       const int slot = first_row ? 0 : 1;
-      // The warp's 32 rows x 128 columns of O leave through its 4 KB staging slot, one block of
-      // 32 rows x 128 bytes at a time (bf16: 64 columns, fp32: 32 columns), written in the
-      // 128-byte-swizzle layout (lane = row, 16-byte chunk c at c ^ (row & 7)) and stored by one
-      // TMA tile store per block; the warp does not wait for the global writes.
-      uint8_t* stg = sY + grp * kXSlot + quad * 4096;
-      const int nblk = whole ? 2 : 4;
+      if (grp < 2) {
+        // Groups 0 and 1 write the CTA's 256 columns of O (128 each) in blocks of 32 rows x 64
+        // columns (bf16 for an uncut row, fp16 normalised partials for a cut one: 128-byte rows),
+        // staged in the 128-byte-swizzle layout (lane = row, chunk c at c ^ (row & 7)), one TMA
+        // tile store per block; the warps do not wait for the global writes.
+        if (!warp_wait(&bar->pv_done[glast % kNB], (glast / kNB) & 1, guard)) break;
+        tc_fence_after();
+        const int ocol = col0 + grp * 128;
+        const bool own_slot = (grp == 1 && xe_held);
+        uint8_t* est = own_slot ? xslot : stg;
+        const int u0 = g + ubase + grp * nblk;   // shared-slot uses (group 1: only if queued)
 #pragma unroll 1
-      for (int blk = 0; blk < nblk; ++blk) {
-        uint32_t w[32];
-        if (whole) {
+        for (int blk = 0; blk < nblk; ++blk) {
+          uint32_t w[32];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             float v[32];
             tmem_ld32(tmem + lane_off + kTmemO + grp * 128 + blk * 64 + half * 32, v);
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              w[16 * half + i] = pack_bf16x2(v[2 * i] * inv_l, v[2 * i + 1] * inv_l);
+              w[16 * half + i] = whole ? pack_bf16x2(v[2 * i] * inv_l, v[2 * i + 1] * inv_l)
+                                       : pack_f16x2(v[2 * i] * inv_l, v[2 * i + 1] * inv_l);
           }
-        } else {
-          float v[32];
-          tmem_ld32(tmem + lane_off + kTmemO + grp * 128 + blk * 32, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i] * inv_l);
-        }
-        if (blk == nblk - 1) {   // every TMEM read of O is done: the next piece may overwrite it
-          tc_fence_before();
-          mbar_arrive(&bar->o_empty);
-        }
-        if (lane == 0) bulk_wait_read_all();   // the slot's last copy or store has read it
-        __syncwarp();
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-              make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (whole) {
-            if (quad * 32 < p.n_heads) tma_store_3d(&tmO, stg, ocol + blk * 64, quad * 32, row);
-          } else {
-            tma_store_2d(&tmPart, stg, ocol + blk * 32, (pair * 2 + slot) * 128 + quad * 32);
+          if (blk == nblk - 1) {   // every TMEM read of O is done: the next piece may overwrite it
+            tc_fence_before();
+            mbar_arrive(&bar->o_empty);
           }
-          bulk_commit();
+          if (own_slot) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+          } else if (!acquire_stage(u0 + blk)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(est + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (whole) {
+              if (quad * 32 < p.n_heads) tma_store_3d(&tmO, est, ocol + blk * 64, quad * 32, row);
+            } else {
+              tma_store_2d(&tmPart, est, ocol + blk * 64, (pair * 2 + slot) * 128 + quad * 32);
+            }
+            bulk_commit();
+          }
+          if (!own_slot) release_stage(u0 + blk);
         }
+        if (!ok) break;
+        if (own_slot) {   // the stores have read the slot: the peer may refill it
+          if (lane == 0) {
+            bulk_wait_read_all();
+            mbar_arrive_remote_relaxed(xempty_remote);
+          }
+          xe_held = false;
+        }
+      } else {
+        mbar_arrive(&bar->o_empty);   // this group reads no O
       }
       if (whole) {
         if (rank == 0 && grp == 0 && p.lse_out && h < p.n_heads)
@@ -615,10 +732,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       } else if (rank == 0 && grp == 0) {
         p.part_lse[(static_cast<size_t>(pair) * 2 + slot) * 128 + h] = lse;
       }
+      ubase += g1_has_tile ? nblk : 2 * nblk;
       ++pc;
       it.next();
     }
-    if (lane == 0) bulk_wait_all();   // every copy this warp sent has landed in the peer
+    if (lane == 0) bulk_wait_all();   // every copy and store this warp issued has completed
   }
 
   // ------------------------------------------------------------------ teardown
@@ -672,13 +790,13 @@ bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_
   const uint32_t box_q[3] = {64, 128, 1};
   const uint64_t d_o[3] = {kC, H, R}, s_o[2] = {kC * 2, H * kC * 2};
   const uint32_t box_o[3] = {64, 32, 1};
-  const uint64_t d_p[2] = {kC, static_cast<uint64_t>(pairs) * 2 * 128}, s_p[1] = {kC * 4};
-  const uint32_t box_p[2] = {32, 32};
+  const uint64_t d_p[2] = {kC, static_cast<uint64_t>(pairs) * 2 * 128}, s_p[1] = {kC * 2};
+  const uint32_t box_p[2] = {64, 32};
   return encode_tiled(&m->kv, bf, 3, kv, d_kv, s_kv, box_kv, sw) &&
          encode_tiled(&m->pe, bf, 3, pe, d_pe, s_pe, box_kv, sw) &&
          encode_tiled(&m->q, bf, 3, qabs, d_q, s_q, box_q, sw) &&
          encode_tiled(&m->o, bf, 3, o_lat, d_o, s_o, box_o, sw) &&
-         encode_tiled(&m->part, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, part_o, d_p, s_p, box_p, sw);
+         encode_tiled(&m->part, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, part_o, d_p, s_p, box_p, sw);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -725,9 +843,9 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineP
         const int slot = (q == plo && pair_begin(total, pairs, q) < R0) ? 1 : 0;
         const size_t base = (static_cast<size_t>(q) * 2 + slot) * 128 + h;
         lse[b] = __ldg(p.part_lse + base);
-        const float* src = p.part_o + base * kC;
+        const __half* src = p.part_o + base * kC;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[b][i] = __ldg(src + lane + 32 * i);
+        for (int i = 0; i < 16; ++i) v[b][i] = __half2float(src[lane + 32 * i]);
       }
     }
     float m_new = mx;

@@ -149,7 +149,7 @@ mla_status mla_prefill_chunk(mla_ctx* ctx, const void* q_latent, void* residual,
  *   status — device int32 or NULL; device-side problems (a start position outside
  *     [0, max_seq_len), a bounded wait that gave up) are recorded there (caller zeroes it).
  * The library uses no memory but its inputs, its outputs and one fixed scratch array of about
- * 8.5 MB that every device loading the library holds until exit.  Limits: rows <= 4096 (more
+ * 4.3 MB that every device loading the library holds until exit.  Limits: rows <= 4096 (more
  * returns MLA_ERR_INVALID_ARG); the split over keys uses at most 16 SM pairs.  The first call on
  * a device sets the array up (address lookup, kernel attribute), so make it before capturing a
  * stream into a graph.  All calls share the array: calls that can overlap on the GPU race and
