@@ -6,6 +6,8 @@ cache L=4096 (keys 0..4096), bf16, synthetic seeded inputs resident in HBM.  Bet
 L2 is flushed by writing a 256 MiB buffer and then reading another 256 MiB buffer (both untimed):
 the step starts with none of its data in L2, and without 126 MB of dirty flush lines that the
 step's own loads and stores would otherwise have to write back (the step's inputs are 261 MB).
+The timed steps replay a CUDA graph of one call on a dedicated stream (--no-graph: the eager
+call); the stage breakdown and the end-to-end number use eager calls through the C ABI.
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
         [--workload v32_decode|kimi_decode|ragged_decode|tiny_decode|prefill_chunk]
@@ -200,7 +202,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     out = torch.empty(out_shape, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
+    # a dedicated stream (the legacy default stream serialises with every other stream and
+    # measured ~6 µs slower per step); torch's flush kernels run on it too
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
 
     def flush_l2(i: int) -> None:
         flush.fill_(float(i))   # evict everything the previous step left in L2 ...
@@ -208,15 +213,29 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
 
     def step():
         if w.mode == "decode":
-            rt.decode(q_latent, start_pos, cache, residual=residual, out=out)
+            rt.decode(q_latent, start_pos, cache, residual=residual, out=out, stream=stream)
         else:
-            rt.prefill(q_latent, w.prefill_start, cache, residual=residual, out=out)
+            rt.prefill(q_latent, w.prefill_start, cache, residual=residual, out=out,
+                       stream=stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    if rt.sync_status() != 0:
+    if rt.sync_status(stream) != 0:
         raise RuntimeError("device status set during warm-up")
+    # The timed steps replay a CUDA graph of one step (the same six kernels with the same
+    # arguments, chained by programmatic dependent launch, without per-call host work); --no-graph
+    # times the eager C-ABI call instead.
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        graph.replay()
+        torch.cuda.synchronize()
+        if rt.sync_status(stream) != 0:
+            raise RuntimeError("device status set by the captured step")
+    run_step = graph.replay if graph is not None else step
 
     # ---- timed region: K steps, L2 flushed before each (flush not timed)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -230,14 +249,14 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     for i in range(args.steps):
         flush_l2(i)
         starts[i].record(stream)
-        step()
+        run_step()
         ends[i].record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
     launches = mla_last_launch_count(rt.ctx)
-    if rt.sync_status() != 0:
+    if rt.sync_status(stream) != 0:
         raise RuntimeError("device status set during the timed steps")
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = float(sum(step_ms))
@@ -269,9 +288,9 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         d_q.copy_(h_q, non_blocking=True)
         d_sp.copy_(h_sp, non_blocking=True)
         if w.mode == "decode":
-            rt.decode(d_q, d_sp, cache, residual=residual, out=out)
+            rt.decode(d_q, d_sp, cache, residual=residual, out=out, stream=stream)
         else:
-            rt.prefill(d_q, w.prefill_start, cache, residual=residual, out=out)
+            rt.prefill(d_q, w.prefill_start, cache, residual=residual, out=out, stream=stream)
         h_out.copy_(out, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
@@ -321,6 +340,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                    "cache_keys_per_step": work["keys"], "q_lora": 1536, "kv_lora": 512,
                    "rope": 64, "v": 128,
                    "l2": "flushed before every timed step: 256 MiB write, then 256 MiB read of another buffer (untimed)",
+                   "launch": "eager C-ABI call" if args.no_graph else "CUDA graph of one C-ABI call, replayed on a dedicated stream",
                    "parallelism": f"replicas x{world} (sequence-sharded, no collective)"},
         "hbm": {"step_bytes": work["bytes"], "step_gbs": round(step_gbs, 1),
                 "frac_of_peak": round(step_gbs / peaks["hbm_gbs"], 4)},
@@ -406,6 +426,8 @@ def main(argv=None):
                     help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--ref-step-seconds", type=float, default=6.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the eager C-ABI call instead of a CUDA-graph replay of it")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
