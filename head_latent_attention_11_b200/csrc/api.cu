@@ -84,7 +84,8 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
-  size_t status, w_ukt, y, rope, q_nope, qabs, o_lat, part_o, part_lse, prefix, pair_row, total;
+  size_t status, w_ukt, y, rope, q_nope, qabs, o_lat, part_o, part_lse, prefix, pair_row,
+      row_pieces, total;
 };
 
 int device_pairs() { return attention_pairs(); }
@@ -129,6 +130,7 @@ Layout layout_of(const mla_config* c) {
   L.part_lse = take(pairs * 2 * 128 * 4);
   L.prefix = take((rows + 1) * 8);
   L.pair_row = take(pairs * 4);
+  L.row_pieces = take(rows * 8);
   L.total = off;
   return L;
 }
@@ -164,6 +166,7 @@ struct mla_ctx {
   float* part_lse() const { return reinterpret_cast<float*>(ws + L.part_lse); }
   long long* prefix() const { return reinterpret_cast<long long*>(ws + L.prefix); }
   int* pair_row() const { return reinterpret_cast<int*>(ws + L.pair_row); }
+  int2* row_pieces() const { return reinterpret_cast<int2*>(ws + L.row_pieces); }
 };
 
 namespace {
@@ -250,6 +253,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   rp.max_seq_len = c->cfg.max_seq_len;
   rp.row_prefix = c->prefix();
   rp.pair_row = c->pair_row();
+  rp.row_pieces = c->row_pieces();
   rp.n_pairs = c->n_pairs;
   rp.min_keys_per_pair = kMinKeysPerPair;
   rp.status = c->status();
@@ -310,7 +314,9 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   MLA_TRY(launch_attention(am, ap, c->n_pairs, s, true));
   ++launches;
 
-  // 5. combine rows cut between pairs
+  // 5. combine rows cut between pairs — for at most 64 rows the W_UV GEMM merges them itself
+  // while it builds its B operand (no separate launch)
+  const bool merge_in_wuv = rows <= 64;
   CombineParams cp{};
   cp.row_prefix = c->prefix();
   cp.rows = rows;
@@ -319,11 +325,14 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   cp.min_keys_per_pair = kMinKeysPerPair;
   cp.part_o = c->part_o();
   cp.part_lse = c->part_lse();
+  cp.row_pieces = c->row_pieces();
   cp.o_lat = c->o_lat();
   cp.lse_out = lse;
-  clk.mark("combine");
-  MLA_TRY(launch_combine(cp, s, true));
-  ++launches;
+  if (!merge_in_wuv) {
+    clk.mark("combine");
+    MLA_TRY(launch_combine(cp, s, true));
+    ++launches;
+  }
 
   // 6. W_UV expansion (one batch per head)
   GemmParams g3{};
@@ -337,6 +346,17 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   g3.ld_g0 = kDv;
   g3.n_heads = H;
   g3.status = c->status();
+  if (merge_in_wuv) {
+    g3.bmerge = 1;
+    g3.row_prefix = c->prefix();
+    g3.part_o = c->part_o();
+    g3.part_lse = c->part_lse();
+    g3.row_pieces = c->row_pieces();
+    g3.o_lat = c->o_lat();
+    g3.lse_out = lse;
+    g3.n_pairs = c->n_pairs;
+    g3.min_keys_per_pair = kMinKeysPerPair;
+  }
   clk.mark("w_uv");
   MLA_TRY(launch_gemm(c->tm_wuv, tm_olat, g3, H, s, true));
   ++launches;

@@ -47,6 +47,9 @@ struct RmsParams {
   // first row of each attention pair's key range (written by block 0 after the prefix);
   // null to skip.  n_pairs / min_keys_per_pair as given to the attention kernel.
   int* pair_row;            // [n_pairs]
+  // per row: the first and last pair its keys fall in, {2 * plo + (plo began in an earlier
+  // row), phi} (written with pair_row; null to skip)
+  int2* row_pieces;         // [rows]
   int n_pairs;
   int min_keys_per_pair;
   int* status;
@@ -70,6 +73,17 @@ struct GemmParams {
   const float2* rope_tab;  // [N, 32]
   int n_heads;
   int* status;
+  // W_UV only, N <= 64 (merge mode): B = o_lat is built in shared memory by the epilogue warps,
+  // merging the attention's split-K pieces of each token (row) for the CTA's head; uncut rows
+  // are read from o_lat, merged rows are written back to o_lat (and lse_out when given).
+  int bmerge;
+  const long long* row_prefix;  // [rows + 1]
+  const __half* part_o;         // [pairs, 2, 128, 512]
+  const float* part_lse;        // [pairs, 2, 128]
+  const int2* row_pieces;       // [rows] see RmsParams::row_pieces
+  bf16* o_lat;                  // [rows, n_heads, 512]
+  float* lse_out;               // [rows, n_heads] or null
+  int n_pairs, min_keys_per_pair;
 };
 
 // ---------------------------------------------------------------------------------------
@@ -103,6 +117,7 @@ struct CombineParams {
   int min_keys_per_pair;
   const __half* part_o;
   const float* part_lse;
+  const int2* row_pieces;       // [rows] see RmsParams::row_pieces
   bf16* o_lat;
   float* lse_out;
 };
@@ -170,6 +185,15 @@ __host__ __device__ inline int active_pairs(long long total_keys, int launched, 
 }
 __host__ __device__ inline long long pair_begin(long long total_keys, int pairs, int p) {
   return total_keys * p / pairs;
+}
+
+// Pair whose key range contains flattened key e.
+__host__ __device__ inline int pair_of_key(long long total, int pairs, long long e) {
+  int q = static_cast<int>((e * pairs) / total);
+  if (q >= pairs) q = pairs - 1;
+  while (q + 1 < pairs && pair_begin(total, pairs, q + 1) <= e) ++q;
+  while (q > 0 && pair_begin(total, pairs, q) > e) --q;
+  return q;
 }
 
 // Row containing flattened key e: largest r with prefix[r] <= e (plain loads: the prefix may

@@ -803,13 +803,6 @@ bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_
 // Combine: rows cut between pairs merge their normalised partials by log-sum-exp weights.
 // One warp per (row, head) task; lane l owns columns l, l+32, ..., l+480.
 // ------------------------------------------------------------------------------------------
-__device__ __forceinline__ int pair_of_key(long long total, int pairs, long long e) {
-  int q = static_cast<int>((e * pairs) / total);
-  if (q >= pairs) q = pairs - 1;
-  while (q + 1 < pairs && pair_begin(total, pairs, q + 1) <= e) ++q;
-  while (q > 0 && pair_begin(total, pairs, q) > e) --q;
-  return q;
-}
 
 // Persistent grid (one block per SM, launched once): each warp walks (row, head) tasks.
 constexpr int kCombineThreads = 512;
@@ -819,13 +812,12 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineP
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (kCombineThreads / 32);
-  const long long total = p.row_prefix[p.rows];
-  const int pairs = active_pairs(total, p.n_pairs, p.min_keys_per_pair);
   for (int task = blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5);
        task < p.rows * p.n_heads; task += warps) {
   const int r = task / p.n_heads, h = task - r * p.n_heads;
-  const long long R0 = p.row_prefix[r], R1 = p.row_prefix[r + 1];
-  const int plo = pair_of_key(total, pairs, R0), phi = pair_of_key(total, pairs, R1 - 1);
+  const int2 pcs = p.row_pieces[r];
+  const int plo = pcs.x >> 1, phi = pcs.y;
+  const int slot_lo = pcs.x & 1;   // the first piece is the tail of a pair begun in an earlier row
   if (plo == phi) continue;   // written by one pair
   // online log-sum-exp merge, four pieces' loads in flight at a time
   constexpr int kBatch = 4;
@@ -840,7 +832,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineP
       const int q = q0 + b;
       lse[b] = -INFINITY;
       if (q <= phi) {
-        const int slot = (q == plo && pair_begin(total, pairs, q) < R0) ? 1 : 0;
+        const int slot = q == plo ? slot_lo : 0;
         const size_t base = (static_cast<size_t>(q) * 2 + slot) * 128 + h;
         lse[b] = __ldg(p.part_lse + base);
         const __half* src = p.part_o + base * kC;

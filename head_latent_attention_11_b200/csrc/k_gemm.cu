@@ -36,9 +36,161 @@ struct GemmTile {
   static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;   // two accumulators
 };
 
-template <int BN, int STAGES>
+// MERGE (W_UV, K = 512): the ring carries only weight slabs; B (the token rows of o_lat, 8 K-slabs)
+// is built once per output tile in a fixed region by the epilogue warps.
+constexpr int kMergeSlabs = kC / 64;
+
+template <int BN, int STAGES, bool MERGE = false>
 constexpr int gemm_smem_bytes() {
-  return 1024 /*align slack*/ + STAGES * (kSlabA + GemmTile<BN>::kSlabB) + 256 /*barriers*/;
+  return 1024 /*align slack*/ + STAGES * kSlabA +
+         (MERGE ? kMergeSlabs * GemmTile<BN>::kSlabB : STAGES * GemmTile<BN>::kSlabB) +
+         256 /*barriers*/;
+}
+
+// Builds B = o_lat[n0 .. n0+BN)[g][0..512) (bf16, K-major, 128-byte swizzle, 8 slabs of BN rows x
+// 64 columns) for head g in shared memory, merging each row's split-K pieces by log-sum-exp
+// weights; merged rows are also written to o_lat (and their lse to lse_out).  128 threads (the
+// epilogue warps); warp w takes rows w, w+4, ... two at a time with all their loads in flight;
+// lane l owns columns 16l .. 16l+15.  The tile's key prefix is read once (one value per lane).
+template <int BN>
+__device__ void build_merged_b(const GemmParams& p, int g, int n0, uint8_t* sBm, int etid) {
+  const int w = etid >> 5, lane = etid & 31;
+  const int slab = lane >> 2, c0 = (lane & 3) * 2;   // this lane's 16 columns: slab, first chunk
+  constexpr int kPieces = 4;                          // pieces of a row loaded per batch
+  constexpr int kPre = (BN + 31) / 32;                // row records per lane
+  int2 pre[kPre];                                     // row_pieces of the tile's rows
+#pragma unroll
+  for (int k = 0; k < kPre; ++k) {
+    const int n = n0 + lane + 32 * k;
+    pre[k] = n < p.N ? p.row_pieces[n] : make_int2(0, 0);
+  }
+  auto pieces_of = [&](int i) -> int2 {   // row_pieces[n0 + i], 0 <= i < BN (warp-uniform i)
+    int2 v = make_int2(0, 0);
+#pragma unroll
+    for (int k = 0; k < kPre; ++k) {
+      const int x = __shfl_sync(0xffffffffu, pre[k].x, i & 31);
+      const int y = __shfl_sync(0xffffffffu, pre[k].y, i & 31);
+      if ((i >> 5) == k) v = make_int2(x, y);
+    }
+    return v;
+  };
+#pragma unroll 1
+  for (int i0 = w; i0 < BN; i0 += 8) {
+    int plo[2], phi[2], nn[2], slot_lo[2];
+    float lse[2][kPieces];
+    uint4 v[2][kPieces][2];
+    // issue every load of both rows (o_lat row, or up to kPieces partial pieces) first
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int i = i0 + 4 * r;
+      nn[r] = n0 + i;
+      plo[r] = 0;
+      phi[r] = -1;
+      const int2 pcs = pieces_of(i < BN ? i : 0);
+      if (i < BN && nn[r] < p.N) {
+        plo[r] = pcs.x >> 1;
+        slot_lo[r] = pcs.x & 1;   // the first piece is the tail of a pair begun in an earlier row
+        phi[r] = pcs.y;
+        const size_t orow = (static_cast<size_t>(nn[r]) * p.n_heads + g) * kC + lane * 16;
+#pragma unroll
+        for (int b = 0; b < kPieces; ++b) {
+          const int q = plo[r] + b;
+          lse[r][b] = -INFINITY;
+          if (plo[r] == phi[r]) {
+            if (b == 0) {   // one piece: the attention kernel wrote this row of o_lat
+              const uint4* src = reinterpret_cast<const uint4*>(p.o_lat + orow);
+              v[r][0][0] = src[0];
+              v[r][0][1] = src[1];
+            }
+          } else if (q <= phi[r]) {
+            const int slot = b == 0 ? slot_lo[r] : 0;
+            const size_t base = (static_cast<size_t>(q) * 2 + slot) * 128 + g;
+            lse[r][b] = p.part_lse[base];
+            const uint4* src = reinterpret_cast<const uint4*>(p.part_o + base * kC + lane * 16);
+            v[r][b][0] = src[0];
+            v[r][b][1] = src[1];
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int i = i0 + 4 * r;
+      if (i >= BN) continue;
+      uint4 out_lo = make_uint4(0, 0, 0, 0), out_hi = make_uint4(0, 0, 0, 0);
+      if (nn[r] < p.N) {
+        if (plo[r] == phi[r]) {
+          out_lo = v[r][0][0];
+          out_hi = v[r][0][1];
+        } else {
+          // online log-sum-exp merge; rows of more than kPieces pieces load the rest here
+          float mx = -INFINITY, wsum = 0.f, acc[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+          for (int q0 = plo[r]; q0 <= phi[r]; q0 += kPieces) {
+            float l_b[kPieces];
+            uint4 v_b[kPieces][2];
+#pragma unroll
+            for (int b = 0; b < kPieces; ++b) {
+              if (q0 == plo[r]) {
+                l_b[b] = lse[r][b];
+                v_b[b][0] = v[r][b][0];
+                v_b[b][1] = v[r][b][1];
+              } else {
+                const int q = q0 + b;
+                l_b[b] = -INFINITY;
+                if (q <= phi[r]) {
+                  const size_t base = static_cast<size_t>(q) * 2 * 128 + g;   // slot 0
+                  l_b[b] = p.part_lse[base];
+                  const uint4* src =
+                      reinterpret_cast<const uint4*>(p.part_o + base * kC + lane * 16);
+                  v_b[b][0] = src[0];
+                  v_b[b][1] = src[1];
+                }
+              }
+            }
+            float m_new = mx;
+#pragma unroll
+            for (int b = 0; b < kPieces; ++b) m_new = fmaxf(m_new, l_b[b]);
+            const float f = mx == -INFINITY ? 0.f : exp2f((mx - m_new) * 1.4426950408889634f);
+            wsum *= f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) acc[k] *= f;
+#pragma unroll
+            for (int b = 0; b < kPieces; ++b) {
+              if (q0 + b <= phi[r]) {
+                const float wt = exp2f((l_b[b] - m_new) * 1.4426950408889634f);
+                wsum += wt;
+                const __half2* hv = reinterpret_cast<const __half2*>(v_b[b]);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  const float2 x = __half22float2(hv[k]);
+                  acc[2 * k] = fmaf(wt, x.x, acc[2 * k]);
+                  acc[2 * k + 1] = fmaf(wt, x.y, acc[2 * k + 1]);
+                }
+              }
+            }
+            mx = m_new;
+          }
+          const float inv = 1.f / wsum;
+          uint32_t o[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) o[k] = pack_bf16x2(acc[2 * k] * inv, acc[2 * k + 1] * inv);
+          out_lo = make_uint4(o[0], o[1], o[2], o[3]);
+          out_hi = make_uint4(o[4], o[5], o[6], o[7]);
+          uint4* dst = reinterpret_cast<uint4*>(
+              p.o_lat + (static_cast<size_t>(nn[r]) * p.n_heads + g) * kC + lane * 16);
+          dst[0] = out_lo;
+          dst[1] = out_hi;
+          if (lane == 0 && p.lse_out)
+            p.lse_out[static_cast<size_t>(nn[r]) * p.n_heads + g] = mx + logf(wsum);
+        }
+      }
+      uint8_t* rowp = sBm + slab * GemmTile<BN>::kSlabB + i * 128;
+      *reinterpret_cast<uint4*>(rowp + ((c0 ^ (i & 7)) << 4)) = out_lo;
+      *reinterpret_cast<uint4*>(rowp + (((c0 + 1) ^ (i & 7)) << 4)) = out_hi;
+    }
+  }
 }
 
 __device__ __forceinline__ void epi_store(const GemmParams& p, int g, int m, int n, float v,
@@ -96,7 +248,7 @@ struct Sched {
   }
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool MERGE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmParams p, const int batches) {
@@ -104,14 +256,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * kSlabA;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * GemmTile<BN>::kSlabB);
+  uint8_t* sB = smem + STAGES * kSlabA;   // MERGE: the tile's 8 B slabs; else the ring's B slabs
+  constexpr int kSmemB = MERGE ? kMergeSlabs * GemmTile<BN>::kSlabB : STAGES * GemmTile<BN>::kSlabB;
+  constexpr uint32_t kStageTx = MERGE ? kSlabA : kSlabA + GemmTile<BN>::kSlabB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kSmemB);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;        // [2]
   uint64_t* acc_empty = bars + 2 * STAGES + 2;   // [2]
   uint64_t* drain = bars + 2 * STAGES + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  uint64_t* b_ready = bars + 2 * STAGES + 5;     // MERGE: the tile's B block is built
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   pdl_launch_dependents();
@@ -134,6 +289,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&acc_empty[i], 128);
     }
     mbar_init(drain, 1);
+    mbar_init(b_ready, 128);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -157,7 +313,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         while (npre < STAGES && pre.next(u)) {
           const Unit un = unit_of(u, mt, nt, BN);
           for (int j = 0; j < nk && npre < STAGES; ++j, ++npre) {
-            mbar_arrive_expect_tx(&full[npre], kSlabA + GemmTile<BN>::kSlabB);
+            mbar_arrive_expect_tx(&full[npre], kStageTx);
             tma_load_3d_hint(sA + npre * kSlabA, &tmA, &full[npre], j * 64, un.m0 + p.a_row_off,
                              un.g, pol_w);
           }
@@ -176,11 +332,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&full[s], kSlabA + GemmTile<BN>::kSlabB);
+            mbar_arrive_expect_tx(&full[s], kStageTx);
             tma_load_3d_hint(sA + s * kSlabA, &tmA, &full[s], j * 64, un.m0 + p.a_row_off, un.g,
                              pol_w);
           }
-          tma_load_3d(sB + s * GemmTile<BN>::kSlabB, &tmB, &full[s], j * 64, un.g, un.n0);
+          if (!MERGE) tma_load_3d(sB + s * GemmTile<BN>::kSlabB, &tmB, &full[s], j * 64, un.g, un.n0);
         }
       }
       if (guard.aborted()) {
@@ -200,6 +356,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       while (ok && sched.next(u)) {
         const int ab = si & 1;
         if (si >= 2 && !mbar_wait(&acc_empty[ab], ((si >> 1) - 1) & 1, guard)) break;
+        if (MERGE && !mbar_wait(b_ready, si & 1, guard)) break;
         tc_fence_after();
         const uint32_t d = tmem + ab * BN;
         for (int j = 0; j < nk; ++j, ++ks) {
@@ -207,7 +364,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!mbar_wait(&full[s], (ks / STAGES) & 1, guard)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * kSlabA);
-          const uint32_t b0 = smem_u32(sB + s * GemmTile<BN>::kSlabB);
+          const uint32_t b0 = smem_u32(sB + (MERGE ? j : s) * GemmTile<BN>::kSlabB);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             umma_bf16(d, smem_desc_sw128(a0 + kk * 32, 16, 1024),
@@ -232,6 +389,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     while (sched.next(u)) {
       const Unit un = unit_of(u, mt, nt, BN);
       const int ab = si & 1;
+      if constexpr (MERGE) {
+        // the previous tile's MMAs have completed (its acc_full was observed): rebuild B
+        build_merged_b<BN>(p, un.g, un.n0, sB, static_cast<int>(threadIdx.x) - 64);
+        fence_async_smem();
+        mbar_arrive(b_ready);
+      }
       if (!warp_wait(&acc_full[ab], (si >> 1) & 1, guard)) break;
       tc_fence_after();
       const int m = un.m0 + row;
@@ -266,7 +429,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 int g_num_sms = 0;
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool MERGE>
 cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                           int batches, cudaStream_t s, bool pdl) {
   if (g_num_sms == 0) {
@@ -277,35 +440,43 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Ge
   }
   const int total = batches * (p.M / 128) * ((p.N + BN - 1) / BN);
   const int grid = total < g_num_sms ? total : g_num_sms;
-  LaunchCfg lc(dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<BN, STAGES>(), s, pdl);
-  return cudaLaunchKernelEx(&lc.cfg, gemm_bf16_kernel<BN, STAGES>, ta, tb, p, batches);
+  LaunchCfg lc(dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<BN, STAGES, MERGE>(), s, pdl);
+  return cudaLaunchKernelEx(&lc.cfg, gemm_bf16_kernel<BN, STAGES, MERGE>, ta, tb, p, batches);
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool MERGE>
 cudaError_t set_attr() {
-  static_assert(gemm_smem_bytes<BN, STAGES>() <= 232448, "shared memory budget");
-  return cudaFuncSetAttribute(gemm_bf16_kernel<BN, STAGES>,
+  static_assert(gemm_smem_bytes<BN, STAGES, MERGE>() <= 232448, "shared memory budget");
+  return cudaFuncSetAttribute(gemm_bf16_kernel<BN, STAGES, MERGE>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              gemm_smem_bytes<BN, STAGES>());
+                              gemm_smem_bytes<BN, STAGES, MERGE>());
 }
 
 }  // namespace
 
 // Tile choice: BN covers the token count up to 256; the ring fills ~200 KB of shared memory.
+// The merge mode (W_UV for at most 64 rows) keeps 8 B slabs resident and a 10/8-stage A ring.
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                         int batches, cudaStream_t s, bool pdl) {
-  if (p.N <= 32) return launch_gemm_t<32, 10>(ta, tb, p, batches, s, pdl);
-  if (p.N <= 64) return launch_gemm_t<64, 8>(ta, tb, p, batches, s, pdl);
-  if (p.N <= 128) return launch_gemm_t<128, 6>(ta, tb, p, batches, s, pdl);
-  return launch_gemm_t<256, 4>(ta, tb, p, batches, s, pdl);
+  if (p.bmerge) {
+    if (p.K != kC || p.N > 64) return cudaErrorInvalidValue;
+    if (p.N <= 32) return launch_gemm_t<32, 10, true>(ta, tb, p, batches, s, pdl);
+    return launch_gemm_t<64, 8, true>(ta, tb, p, batches, s, pdl);
+  }
+  if (p.N <= 32) return launch_gemm_t<32, 10, false>(ta, tb, p, batches, s, pdl);
+  if (p.N <= 64) return launch_gemm_t<64, 8, false>(ta, tb, p, batches, s, pdl);
+  if (p.N <= 128) return launch_gemm_t<128, 6, false>(ta, tb, p, batches, s, pdl);
+  return launch_gemm_t<256, 4, false>(ta, tb, p, batches, s, pdl);
 }
 
 cudaError_t gemm_prepare() {
   cudaError_t e;
-  if ((e = set_attr<32, 10>()) != cudaSuccess) return e;
-  if ((e = set_attr<64, 8>()) != cudaSuccess) return e;
-  if ((e = set_attr<128, 6>()) != cudaSuccess) return e;
-  return set_attr<256, 4>();
+  if ((e = set_attr<32, 10, false>()) != cudaSuccess) return e;
+  if ((e = set_attr<64, 8, false>()) != cudaSuccess) return e;
+  if ((e = set_attr<128, 6, false>()) != cudaSuccess) return e;
+  if ((e = set_attr<256, 4, false>()) != cudaSuccess) return e;
+  if ((e = set_attr<32, 10, true>()) != cudaSuccess) return e;
+  return set_attr<64, 8, true>();
 }
 
 // W_UK^T copy made once at set-up: w_ukt[h][c][d] = wkv_b[h*256 + d][c], d < 128, so that the

@@ -68,8 +68,17 @@ __device__ void key_prefix_block(const RmsParams& p) {
     acc += row_position(p, r, &bad) + 1;
     p.row_prefix[r + 1] = acc;
     if (p.pair_row) {
-      const long long q1 = first_pair_at(acc) < pairs ? first_pair_at(acc) : pairs;
-      for (long long q = first_pair_at(R0); q < q1; ++q) p.pair_row[q] = r;
+      const long long qa = first_pair_at(R0), qb = first_pair_at(acc);
+      const long long q1 = qb < pairs ? qb : pairs;
+      for (long long q = qa; q < q1; ++q) p.pair_row[q] = r;
+      if (p.row_pieces) {
+        // pair qa begins at or after R0; it begins exactly there iff total*qa < (R0+1)*pairs.
+        // Otherwise the row's first key belongs to pair qa-1, which began in an earlier row.
+        const bool starts_here = qa < pairs && total * qa < (R0 + 1) * pairs;
+        const int plo = static_cast<int>(starts_here ? qa : qa - 1);
+        const int phi = static_cast<int>(q1 - 1);
+        p.row_pieces[r] = make_int2(2 * plo + (starts_here ? 0 : 1), phi);
+      }
     }
   }
   if (bad) atomicCAS(p.status, kDevOk, kDevBadArg);

@@ -31,7 +31,8 @@ constexpr size_t kOffPrefix = 256;
 constexpr size_t kOffPartO = kOffPrefix + ((static_cast<size_t>(kNoAllocMaxRows) + 1) * 8 + 255) / 256 * 256;
 constexpr size_t kOffPartLse = kOffPartO + static_cast<size_t>(kNoAllocPairs) * 2 * 128 * kC * 2;
 constexpr size_t kOffPairRow = kOffPartLse + static_cast<size_t>(kNoAllocPairs) * 2 * 128 * 4;
-constexpr size_t kScratchBytes = kOffPairRow + 256;
+constexpr size_t kOffRowPieces = kOffPairRow + 256;
+constexpr size_t kScratchBytes = kOffRowPieces + static_cast<size_t>(kNoAllocMaxRows) * 8;
 
 // ~4.3 MB on every device that loads the library, kept until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
@@ -88,6 +89,7 @@ extern "C" mla_status mla_latent_attention_noalloc(
   __half* part_o = reinterpret_cast<__half*>(scratch + kOffPartO);
   float* part_lse = reinterpret_cast<float*>(scratch + kOffPartLse);
   int* pair_row = reinterpret_cast<int*>(scratch + kOffPairRow);
+  int2* row_pieces = reinterpret_cast<int2*>(scratch + kOffRowPieces);
 
   const int pairs = attention_pairs() < kNoAllocPairs ? attention_pairs() : kNoAllocPairs;
   AttnMaps am;
@@ -106,6 +108,7 @@ extern "C" mla_status mla_latent_attention_noalloc(
   rp.max_seq_len = max_seq_len;
   rp.row_prefix = prefix;
   rp.pair_row = pair_row;
+  rp.row_pieces = row_pieces;
   rp.n_pairs = pairs;
   rp.min_keys_per_pair = 256;
   rp.status = st;
@@ -137,6 +140,7 @@ extern "C" mla_status mla_latent_attention_noalloc(
   cp.min_keys_per_pair = 256;
   cp.part_o = part_o;
   cp.part_lse = part_lse;
+  cp.row_pieces = row_pieces;
   cp.o_lat = static_cast<bf16*>(o_lat);
   cp.lse_out = lse;
   if (launch_combine(cp, stream, false) != cudaSuccess) return MLA_ERR_CUDA;
