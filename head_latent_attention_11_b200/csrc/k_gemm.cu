@@ -193,8 +193,25 @@ __device__ void build_merged_b(const GemmParams& p, int g, int n0, uint8_t* sBm,
   }
 }
 
+// The rotary (cos, sin) of row m's pair for tokens n0 .. n0+15, all loads issued before any
+// store of the block (a store between them would keep each load waiting for the one before).
+__device__ __forceinline__ void rope_prefetch(const GemmParams& p, int m, int n0, float2 (&cs)[16]) {
+  const int h = m / kDq, j = m - h * kDq;
+  if (p.epi != kEpiWqbRope || j < kDn) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) cs[i] = make_float2(1.f, 0.f);   // unused outside the rope rows
+    return;
+  }
+  const int pair = (j - kDn) >> 1;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int n = n0 + i < p.N ? n0 + i : p.N - 1;
+    cs[i] = __ldg(p.rope_tab + static_cast<size_t>(n) * kRopePairs + pair);
+  }
+}
+
 __device__ __forceinline__ void epi_store(const GemmParams& p, int g, int m, int n, float v,
-                                          float partner) {
+                                          float partner, float2 cs) {
   if (p.epi == kEpiWqbRope) {
     const int h = m / kDq, j = m - h * kDq;
     if (j < kDn) {
@@ -202,7 +219,6 @@ __device__ __forceinline__ void epi_store(const GemmParams& p, int g, int m, int
           __float2bfloat16_rn(v);
     } else {
       const int jj = j - kDn;                 // 0..63, pair jj/2
-      const float2 cs = p.rope_tab[static_cast<size_t>(n) * kRopePairs + (jj >> 1)];
       // q is a bf16 tensor before the rotation (bf16 wq_b output, "Query heads" mla-queries)
       v = bf16_round(v);
       partner = bf16_round(partner);
@@ -232,7 +248,7 @@ __device__ __forceinline__ Unit unit_of(int u, int mt, int nt, int BN) {
   return r;
 }
 
-// Work split: CTA c takes units c, c + G, c + 2G, ... (G = grid size).
+// Work split: CTA c takes output tiles c, c + G, c + 2G, ... (G = grid size).
 struct Sched {
   int units, G, u;
   __device__ void init(int nunits, int grid, int cta) {
@@ -384,6 +400,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int quad = warp & 3;
     const int row = quad * 32 + static_cast<int>(lane_id());
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const int etid = static_cast<int>(threadIdx.x) - 64;   // 0..127
     int si = 0;
     int u;
     while (sched.next(u)) {
@@ -391,7 +408,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int ab = si & 1;
       if constexpr (MERGE) {
         // the previous tile's MMAs have completed (its acc_full was observed): rebuild B
-        build_merged_b<BN>(p, un.g, un.n0, sB, static_cast<int>(threadIdx.x) - 64);
+        build_merged_b<BN>(p, un.g, un.n0, sB, etid);
         fence_async_smem();
         mbar_arrive(b_ready);
       }
@@ -402,12 +419,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int c0 = 0; c0 < BN; c0 += 16) {
         if (un.n0 + c0 >= p.N) break;   // uniform across the warp
         float v[16];
+        float2 cs[16];
+        rope_prefetch(p, m, un.n0 + c0, cs);
         tmem_ld16(tmem + lane_off + ab * BN + c0, v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float partner = __shfl_xor_sync(0xffffffffu, v[i], 1);
           const int n = un.n0 + c0 + i;
-          if (n < p.N) epi_store(p, un.g, m, n, v[i], partner);
+          if (n < p.N) epi_store(p, un.g, m, n, v[i], partner, cs[i]);
         }
       }
       tc_fence_before();
