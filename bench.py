@@ -114,54 +114,106 @@ def aggregate_throughput(units_per_rank: int, steps: int, world: int, max_ms: fl
 # Clock sampling during the timed region
 # ------------------------------------------------------------------------------------------
 class ClockSampler:
+    """Samples the SM clock and the clock-event reasons of one GPU from a background thread.
+
+    NVML is polled every 5 ms (read-only queries); where NVML is unavailable, nvidia-smi's
+    100 ms loop is used instead.  `mark(name)` stamps host times so that the summary can say
+    how many samples fell inside the timed region proper."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.samples: list[tuple[float, float, set]] = []   # (host time, SM MHz, reasons)
+        self.sm_max = None
+        self.marks: dict[str, float] = {}
+        self.source = None
+        self._stop = threading.Event()
+        self._t = None
         self.proc = None
-        self.lines: list[str] = []
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+        h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        return pynvml, h
 
     def start(self):
         try:
+            nv, h = self._nvml_handle()
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            self.sm_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+
+            def poll():
+                while not self._stop.is_set():
+                    mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    mask = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((time.perf_counter(), mhz,
+                                         {n for n, b in bits.items() if mask & b}))
+                    time.sleep(0.005)
+
+            self.source = "nvml, 5 ms"
+            self._t = threading.Thread(target=poll, daemon=True)
+            self._t.start()
+            return
+        except Exception:
+            pass
+        try:
+            gpu = os.environ.get("CUDA_VISIBLE_DEVICES", str(self.dev)).split(",")[self.dev] or "0"
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", "-i", gpu, f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self._t = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi, 100 ms"
+            self._t = threading.Thread(target=self._read_smi, daemon=True)
             self._t.start()
-        except (FileNotFoundError, OSError):
+        except (FileNotFoundError, OSError, IndexError):
             self.proc = None
 
-    def _read(self):
+    def _read_smi(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
+            parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
+                mhz, self.sm_max = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+            self.samples.append((time.perf_counter(), mhz,
+                                 {n for n, v in zip(self.REASONS, parts[5:9]) if v.lower() == "active"}))
+
+    def mark(self, name: str) -> None:
+        self.marks[name] = time.perf_counter()
+
+    def stop(self) -> dict:
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock query unavailable"]}
+        self._stop.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self._t is not None:
+            self._t.join(timeout=5)
+        lo = self.marks.get("load", float("-inf"))
+        t0, t1 = self.marks.get("timed0", lo), self.marks.get("timed1", float("inf"))
+        under_load = [s for s in self.samples if lo <= s[0] <= t1]
+        timed = [s for s in under_load if s[0] >= t0]
+        reasons = set().union(*[s[2] for s in under_load]) if under_load else set()
+        return {"sm_mhz": statistics.median([s[1] for s in under_load]) if under_load else None,
+                "sm_max_mhz": self.sm_max, "reasons": sorted(reasons),
+                "samples": len(under_load), "samples_timed": len(timed),
+                "source": self.source,
+                "window": "untimed load steps (0.5 s) directly before the timed steps, then the timed steps"}
 
 
 # ------------------------------------------------------------------------------------------
@@ -240,18 +292,28 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     # ---- timed region: K steps, L2 flushed before each (flush not timed)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    clocks = ClockSampler(local_rank if world > 1 else int(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or 0))
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    # keep the GPU busy for ~0.5 s right before the timed steps (same flush + step, untimed) so
+    # that the clock record holds enough samples taken under this load
+    clocks.mark("load")
+    t_load = time.perf_counter()
+    while time.perf_counter() - t_load < 0.5:
+        for i in range(32):
+            flush_l2(i)
+            run_step()
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
+    clocks.mark("timed0")
     for i in range(args.steps):
         flush_l2(i)
         starts[i].record(stream)
         run_step()
         ends[i].record(stream)
     torch.cuda.synchronize()
+    clocks.mark("timed1")
     if world > 1:
         dist.barrier()
     clk = clocks.stop()

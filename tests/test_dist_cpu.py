@@ -49,3 +49,19 @@ def test_single_process_is_identity():
     import bench
     assert bench.max_over_ranks([1.5, 2.5]) == [1.5, 2.5]
     assert bench.aggregate_throughput(32, 4, 1, 8.0) == pytest.approx(16000.0)
+
+
+def test_clock_record_counts_only_loaded_samples():
+    """The clock summary takes the median over the load window and the timed steps, ignores
+    samples taken before the load started, and reports every throttle reason seen under load."""
+    import bench
+    c = bench.ClockSampler(0)
+    c.source, c.sm_max = "test", 1965.0
+    c.samples = [(0.0, 345.0, set()), (1.0, 1965.0, set()), (1.1, 1900.0, {"sw_power_cap"}),
+                 (1.2, 1965.0, set()), (1.3, 1950.0, set()), (9.0, 300.0, {"hw_slowdown"})]
+    c.marks = {"load": 0.5, "timed0": 1.15, "timed1": 1.35}
+    r = c.stop()
+    assert r["samples"] == 4 and r["samples_timed"] == 2
+    assert r["sm_mhz"] == pytest.approx(1957.5)
+    assert r["reasons"] == ["sw_power_cap"]
+    assert r["sm_max_mhz"] == 1965.0
