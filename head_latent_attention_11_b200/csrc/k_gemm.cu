@@ -40,11 +40,15 @@ struct GemmTile {
 // is built once per output tile in a fixed region by the epilogue warps.
 constexpr int kMergeSlabs = kC / 64;
 
+// Plain-store epilogue: each epilogue warp transposes its 32 rows x 16 tokens of bf16 through a
+// 1 KB staging block so that the global writes are 16-byte vectors.
+constexpr int kEpiStageBytes = 4 * 32 * 16 * 2;
+
 template <int BN, int STAGES, bool MERGE = false>
 constexpr int gemm_smem_bytes() {
   return 1024 /*align slack*/ + STAGES * kSlabA +
          (MERGE ? kMergeSlabs * GemmTile<BN>::kSlabB : STAGES * GemmTile<BN>::kSlabB) +
-         256 /*barriers*/;
+         256 /*barriers*/ + kEpiStageBytes;
 }
 
 // Builds B = o_lat[n0 .. n0+BN)[g][0..512) (bf16, K-major, 128-byte swizzle, 8 slabs of BN rows x
@@ -284,6 +288,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* b_ready = bars + 2 * STAGES + 5;     // MERGE: the tile's B block is built
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* sEpi = reinterpret_cast<uint8_t*>(bars) + 256;   // plain-store epilogue staging
 
   pdl_launch_dependents();
   const int warp = warp_id();
@@ -401,6 +406,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row = quad * 32 + static_cast<int>(lane_id());
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int etid = static_cast<int>(threadIdx.x) - 64;   // 0..127
+    // the plain-store epilogue writes 16-byte vectors when every row start is 16-byte aligned
+    const bool vec_store = p.epi == kEpiStore &&
+                           (reinterpret_cast<uintptr_t>(p.out0) & 15) == 0 &&
+                           (p.ld_n0 & 7) == 0 && (p.ld_g0 & 7) == 0;
     int si = 0;
     int u;
     while (sched.next(u)) {
@@ -415,6 +424,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!warp_wait(&acc_full[ab], (si >> 1) & 1, guard)) break;
       tc_fence_after();
       const int m = un.m0 + row;
+      if (vec_store) {
+        // 16-token blocks: lane = row, value i = token; bf16 into this warp's staging block as
+        // [token][32 rows], then each lane writes two 16-byte pieces (8 rows of one token)
+        __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sEpi + (warp & 3) * 1024);
+        bf16* obase = p.out0 + static_cast<size_t>(un.g) * p.ld_g0 + un.m0 + quad * 32;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          if (un.n0 + c0 >= p.N) break;   // uniform across the warp
+          float v[16];
+          tmem_ld16(tmem + lane_off + ab * BN + c0, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) stg[i * 32 + lane_id()] = __float2bfloat16_rn(v[i]);
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int c = static_cast<int>(lane_id()) + 32 * j;   // 64 pieces of 16 bytes
+            const int t = c >> 2, part = c & 3;
+            const int n = un.n0 + c0 + t;
+            if (n < p.N)
+              *reinterpret_cast<uint4*>(obase + static_cast<size_t>(n) * p.ld_n0 + part * 8) =
+                  *reinterpret_cast<const uint4*>(stg + t * 32 + part * 8);
+          }
+          __syncwarp();   // the block is read before the next one overwrites it
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[ab]);
+        ++si;
+        continue;
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 16) {
         if (un.n0 + c0 >= p.N) break;   // uniform across the warp
