@@ -237,6 +237,31 @@ __device__ __forceinline__ void epi_store(const GemmParams& p, int g, int m, int
   }
 }
 
+// The value the epilogue stores for accumulator row m (same arithmetic as epi_store).
+__device__ __forceinline__ float epi_value(const GemmParams& p, int m, float v, float partner,
+                                           float2 cs) {
+  if (p.epi == kEpiWqbRope) {
+    const int j = m % kDq;
+    if (j >= kDn) {
+      v = bf16_round(v);
+      partner = bf16_round(partner);
+      return ((j - kDn) & 1) == 0 ? v * cs.x - partner * cs.y : partner * cs.y + v * cs.x;
+    }
+  }
+  return v;
+}
+
+// Destination of the 8 consecutive accumulator rows m8 .. m8+7 (m8 a multiple of 8) for token n:
+// 8 consecutive elements, since heads (192 rows) and their content part (128) are multiples of 8.
+__device__ __forceinline__ bf16* epi_dst8(const GemmParams& p, int g, int m8, int n) {
+  if (p.epi == kEpiWqbRope) {
+    const int h = m8 / kDq, j = m8 - h * kDq;
+    if (j < kDn) return p.out0 + static_cast<size_t>(n) * p.ld_n0 + static_cast<size_t>(h) * kDn + j;
+    return p.out1 + (static_cast<size_t>(n) * kHPad + h) * kDk + kC + (j - kDn);
+  }
+  return p.out0 + static_cast<size_t>(n) * p.ld_n0 + static_cast<size_t>(g) * p.ld_g0 + m8;
+}
+
 struct Unit {
   int g, m0, n0;
 };
@@ -406,10 +431,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row = quad * 32 + static_cast<int>(lane_id());
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int etid = static_cast<int>(threadIdx.x) - 64;   // 0..127
-    // the plain-store epilogue writes 16-byte vectors when every row start is 16-byte aligned
-    const bool vec_store = p.epi == kEpiStore &&
-                           (reinterpret_cast<uintptr_t>(p.out0) & 15) == 0 &&
-                           (p.ld_n0 & 7) == 0 && (p.ld_g0 & 7) == 0;
+    // the epilogue writes 16-byte vectors when every 8-row group starts 16-byte aligned
+    const bool vec_store =
+        (reinterpret_cast<uintptr_t>(p.out0) & 15) == 0 && (p.ld_n0 & 7) == 0 &&
+        (p.epi == kEpiStore ? (p.ld_g0 & 7) == 0
+                            : (reinterpret_cast<uintptr_t>(p.out1) & 15) == 0);
     int si = 0;
     int u;
     while (sched.next(u)) {
@@ -428,14 +454,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // 16-token blocks: lane = row, value i = token; bf16 into this warp's staging block as
         // [token][32 rows], then each lane writes two 16-byte pieces (8 rows of one token)
         __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sEpi + (warp & 3) * 1024);
-        bf16* obase = p.out0 + static_cast<size_t>(un.g) * p.ld_g0 + un.m0 + quad * 32;
+        const int mw = un.m0 + quad * 32;   // first row of this warp
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
           if (un.n0 + c0 >= p.N) break;   // uniform across the warp
           float v[16];
+          float2 cs[16];
+          rope_prefetch(p, m, un.n0 + c0, cs);
           tmem_ld16(tmem + lane_off + ab * BN + c0, v);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) stg[i * 32 + lane_id()] = __float2bfloat16_rn(v[i]);
+          for (int i = 0; i < 16; ++i) {
+            const float partner = __shfl_xor_sync(0xffffffffu, v[i], 1);
+            stg[i * 32 + lane_id()] = __float2bfloat16_rn(epi_value(p, m, v[i], partner, cs[i]));
+          }
           __syncwarp();
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
@@ -443,7 +474,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int t = c >> 2, part = c & 3;
             const int n = un.n0 + c0 + t;
             if (n < p.N)
-              *reinterpret_cast<uint4*>(obase + static_cast<size_t>(n) * p.ld_n0 + part * 8) =
+              *reinterpret_cast<uint4*>(epi_dst8(p, un.g, mw + part * 8, n)) =
                   *reinterpret_cast<const uint4*>(stg + t * 32 + part * 8);
           }
           __syncwarp();   // the block is read before the next one overwrites it
