@@ -18,8 +18,10 @@
 //               two accumulators (units alternate), committing each slab back to the producer
 //               and each finished unit to the epilogue;
 //   warps 2-5   epilogue: tcgen05.ld the fp32 accumulator (thread = weight row), apply RoPE for
-//               the rotary rows of wq_b (partner of a pair = neighbouring lane), store bf16,
-//               hand the accumulator back — overlapping the next unit's MMAs.
+//               the rotary rows of wq_b (partner of a pair = neighbouring lane), transpose 16
+//               tokens at a time through shared memory and store bf16 as 16-byte vectors (8
+//               consecutive rows of one token), hand the accumulator back — overlapping the next
+//               unit's MMAs.
 #include "internal.h"
 #include "tc100.cuh"
 
@@ -214,30 +216,9 @@ __device__ __forceinline__ void rope_prefetch(const GemmParams& p, int m, int n0
   }
 }
 
-__device__ __forceinline__ void epi_store(const GemmParams& p, int g, int m, int n, float v,
-                                          float partner, float2 cs) {
-  if (p.epi == kEpiWqbRope) {
-    const int h = m / kDq, j = m - h * kDq;
-    if (j < kDn) {
-      p.out0[static_cast<size_t>(n) * p.ld_n0 + static_cast<size_t>(h) * kDn + j] =
-          __float2bfloat16_rn(v);
-    } else {
-      const int jj = j - kDn;                 // 0..63, pair jj/2
-      // q is a bf16 tensor before the rotation (bf16 wq_b output, "Query heads" mla-queries)
-      v = bf16_round(v);
-      partner = bf16_round(partner);
-      float r;
-      if ((jj & 1) == 0) r = v * cs.x - partner * cs.y;      // x0 cos - x1 sin
-      else r = partner * cs.y + v * cs.x;                     // x0 sin + x1 cos
-      p.out1[(static_cast<size_t>(n) * kHPad + h) * kDk + kC + jj] = __float2bfloat16_rn(r);
-    }
-  } else {
-    p.out0[static_cast<size_t>(n) * p.ld_n0 + static_cast<size_t>(g) * p.ld_g0 + m] =
-        __float2bfloat16_rn(v);
-  }
-}
-
-// The value the epilogue stores for accumulator row m (same arithmetic as epi_store).
+// The value the epilogue stores for accumulator row m: the accumulator itself, or for the rotary
+// rows of wq_b the rotated pair ("Query heads" mla-queries: q is a bf16 tensor before the
+// rotation, so both inputs are rounded to bf16 first).
 __device__ __forceinline__ float epi_value(const GemmParams& p, int m, float v, float partner,
                                            float2 cs) {
   if (p.epi == kEpiWqbRope) {
@@ -431,11 +412,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row = quad * 32 + static_cast<int>(lane_id());
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int etid = static_cast<int>(threadIdx.x) - 64;   // 0..127
-    // the epilogue writes 16-byte vectors when every 8-row group starts 16-byte aligned
-    const bool vec_store =
+    // the epilogue writes 16-byte vectors: every 8-row group must start 16-byte aligned (the C
+    // ABI requires aligned outputs; a violation is reported, never written)
+    const bool aligned_out =
         (reinterpret_cast<uintptr_t>(p.out0) & 15) == 0 && (p.ld_n0 & 7) == 0 &&
         (p.epi == kEpiStore ? (p.ld_g0 & 7) == 0
                             : (reinterpret_cast<uintptr_t>(p.out1) & 15) == 0);
+    if (!aligned_out && etid == 0) guard.fail(kDevBadArg);
     int si = 0;
     int u;
     while (sched.next(u)) {
@@ -450,40 +433,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!warp_wait(&acc_full[ab], (si >> 1) & 1, guard)) break;
       tc_fence_after();
       const int m = un.m0 + row;
-      if (vec_store) {
-        // 16-token blocks: lane = row, value i = token; bf16 into this warp's staging block as
-        // [token][32 rows], then each lane writes two 16-byte pieces (8 rows of one token)
-        __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sEpi + (warp & 3) * 1024);
-        const int mw = un.m0 + quad * 32;   // first row of this warp
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          if (un.n0 + c0 >= p.N) break;   // uniform across the warp
-          float v[16];
-          float2 cs[16];
-          rope_prefetch(p, m, un.n0 + c0, cs);
-          tmem_ld16(tmem + lane_off + ab * BN + c0, v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float partner = __shfl_xor_sync(0xffffffffu, v[i], 1);
-            stg[i * 32 + lane_id()] = __float2bfloat16_rn(epi_value(p, m, v[i], partner, cs[i]));
-          }
-          __syncwarp();
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int c = static_cast<int>(lane_id()) + 32 * j;   // 64 pieces of 16 bytes
-            const int t = c >> 2, part = c & 3;
-            const int n = un.n0 + c0 + t;
-            if (n < p.N)
-              *reinterpret_cast<uint4*>(epi_dst8(p, un.g, mw + part * 8, n)) =
-                  *reinterpret_cast<const uint4*>(stg + t * 32 + part * 8);
-          }
-          __syncwarp();   // the block is read before the next one overwrites it
-        }
-        tc_fence_before();
-        mbar_arrive(&acc_empty[ab]);
-        ++si;
-        continue;
-      }
+      if (!aligned_out) break;
+      // 16-token blocks: lane = row, value i = token; bf16 into this warp's staging block as
+      // [token][32 rows], then each lane writes two 16-byte pieces (8 rows of one token)
+      __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sEpi + (warp & 3) * 1024);
+      const int mw = un.m0 + quad * 32;   // first row of this warp
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 16) {
         if (un.n0 + c0 >= p.N) break;   // uniform across the warp
@@ -494,9 +448,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float partner = __shfl_xor_sync(0xffffffffu, v[i], 1);
-          const int n = un.n0 + c0 + i;
-          if (n < p.N) epi_store(p, un.g, m, n, v[i], partner, cs[i]);
+          stg[i * 32 + lane_id()] = __float2bfloat16_rn(epi_value(p, m, v[i], partner, cs[i]));
         }
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int c = static_cast<int>(lane_id()) + 32 * j;   // 64 pieces of 16 bytes
+          const int t = c >> 2, part = c & 3;
+          const int n = un.n0 + c0 + t;
+          if (n < p.N)
+            *reinterpret_cast<uint4*>(epi_dst8(p, un.g, mw + part * 8, n)) =
+                *reinterpret_cast<const uint4*>(stg + t * 32 + part * 8);
+        }
+        __syncwarp();   // the block is read before the next one overwrites it
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[ab]);

@@ -86,6 +86,30 @@ __device__ void key_prefix_block(const RmsParams& p) {
 
 template <int NCH>
 __global__ void __launch_bounds__(128) rmsnorm_kernel(const RmsParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 4 + warp;
+  const bool live = row < p.rows;
+  // The row's loads go out first, so that block 0's key prefix (its own round trip to memory)
+  // overlaps them instead of preceding them.  The gain is preloaded too when it fits.
+  constexpr bool kPreGain = NCH <= 8;
+  uint4 xv[NCH], rv[NCH];
+  float4 gv[kPreGain ? 2 * NCH : 1];
+  const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(row) * p.dim);
+  uint4* rr = p.residual ? reinterpret_cast<uint4*>(p.residual + static_cast<size_t>(row) * p.dim)
+                         : nullptr;
+  const float4* g4 = reinterpret_cast<const float4*>(p.gamma);
+  if (live) {
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int idx = lane + 32 * c;
+      xv[c] = xr[idx];
+      if (rr) rv[c] = rr[idx];
+      if constexpr (kPreGain) {
+        gv[2 * c] = g4[2 * idx];
+        gv[2 * c + 1] = g4[2 * idx + 1];
+      }
+    }
+  }
   // The kernels after this one start early (programmatic dependent launch) and the attention
   // kernel reads the key prefix before it waits for its predecessors: block 0 therefore writes
   // the prefix first and makes it visible before any block lets the next kernel start.
@@ -95,24 +119,17 @@ __global__ void __launch_bounds__(128) rmsnorm_kernel(const RmsParams p) {
     __syncthreads();
   }
   pdl_launch_dependents();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 4 + warp;
-  if (row < p.rows) {
-    const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(row) * p.dim);
-    uint4* rr = p.residual ? reinterpret_cast<uint4*>(p.residual + static_cast<size_t>(row) * p.dim)
-                           : nullptr;
+  if (live) {
     float u[NCH][8];
     float ss = 0.f;
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
       const int idx = lane + 32 * c;
-      uint4 xv = xr[idx];
-      const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(&xv);
+      const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(&xv[c]);
 #pragma unroll
       for (int i = 0; i < 8; ++i) u[c][i] = __bfloat162float(xb[i]);
       if (rr) {
-        uint4 rv = rr[idx];
-        const __nv_bfloat16* rb = reinterpret_cast<const __nv_bfloat16*>(&rv);
+        const __nv_bfloat16* rb = reinterpret_cast<const __nv_bfloat16*>(&rv[c]);
         uint4 ov;
         uint32_t* o32 = reinterpret_cast<uint32_t*>(&ov);
 #pragma unroll
@@ -128,11 +145,17 @@ __global__ void __launch_bounds__(128) rmsnorm_kernel(const RmsParams p) {
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float inv = rsqrtf(ss / static_cast<float>(p.dim) + p.eps);
     uint4* yr = reinterpret_cast<uint4*>(p.y + static_cast<size_t>(row) * p.dim);
-    const float4* g4 = reinterpret_cast<const float4*>(p.gamma);
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
       const int idx = lane + 32 * c;
-      const float4 ga = g4[2 * idx], gb = g4[2 * idx + 1];
+      float4 ga, gb;
+      if constexpr (kPreGain) {
+        ga = gv[2 * c];
+        gb = gv[2 * c + 1];
+      } else {
+        ga = g4[2 * idx];
+        gb = g4[2 * idx + 1];
+      }
       const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
       uint4 ov;
       uint32_t* o32 = reinterpret_cast<uint32_t*>(&ov);
