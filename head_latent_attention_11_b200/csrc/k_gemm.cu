@@ -17,7 +17,8 @@
 //   warp 1      allocates TMEM and issues tcgen05.mma (M=128, N=BN, K=16) per slab into one of
 //               two accumulators (units alternate), committing each slab back to the producer
 //               and each finished unit to the epilogue;
-//   warps 2-5   epilogue: tcgen05.ld the fp32 accumulator (thread = weight row), apply RoPE for
+//   warps 2-9   epilogue, two warps per TMEM lane quadrant (warp % 4) splitting the 16-token
+//               blocks: tcgen05.ld the fp32 accumulator (thread = weight row), apply RoPE for
 //               the rotary rows of wq_b (partner of a pair = neighbouring lane), transpose 16
 //               tokens at a time through shared memory and store bf16 as 16-byte vectors (8
 //               consecutive rows of one token), hand the accumulator back — overlapping the next
@@ -29,7 +30,9 @@ namespace mla {
 
 namespace {
 
-constexpr int kGemmThreads = 192;
+constexpr int kEpiWarps = 8;                            // two per TMEM lane quadrant
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kGemmThreads = 64 + kEpiThreads;
 constexpr int kSlabA = 128 * 64 * 2;   // 16 KB
 
 template <int BN>
@@ -44,7 +47,7 @@ constexpr int kMergeSlabs = kC / 64;
 
 // Plain-store epilogue: each epilogue warp transposes its 32 rows x 16 tokens of bf16 through a
 // 1 KB staging block so that the global writes are 16-byte vectors.
-constexpr int kEpiStageBytes = 4 * 32 * 16 * 2;
+constexpr int kEpiStageBytes = kEpiWarps * 32 * 16 * 2;
 
 template <int BN, int STAGES, bool MERGE = false>
 constexpr int gemm_smem_bytes() {
@@ -55,14 +58,15 @@ constexpr int gemm_smem_bytes() {
 
 // Builds B = o_lat[n0 .. n0+BN)[g][0..512) (bf16, K-major, 128-byte swizzle, 8 slabs of BN rows x
 // 64 columns) for head g in shared memory, merging each row's split-K pieces by log-sum-exp
-// weights; merged rows are also written to o_lat (and their lse to lse_out).  128 threads (the
-// epilogue warps); warp w takes rows w, w+4, ... two at a time with all their loads in flight;
+// weights; merged rows are also written to o_lat (and their lse to lse_out).  The epilogue warps
+// (kEpiWarps) share the rows: warp w takes rows w, w+kEpiWarps, ... two at a time with all their
+// loads in flight (the merge is a chain of dependent steps per row, so more warps hide more);
 // lane l owns columns 16l .. 16l+15.  The tile's key prefix is read once (one value per lane).
 template <int BN>
 __device__ void build_merged_b(const GemmParams& p, int g, int n0, uint8_t* sBm, int etid) {
   const int w = etid >> 5, lane = etid & 31;
   const int slab = lane >> 2, c0 = (lane & 3) * 2;   // this lane's 16 columns: slab, first chunk
-  constexpr int kPieces = 4;                          // pieces of a row loaded per batch
+  constexpr int kPieces = 3;                          // pieces of a row loaded per batch
   constexpr int kPre = (BN + 31) / 32;                // row records per lane
   int2 pre[kPre];                                     // row_pieces of the tile's rows
 #pragma unroll
@@ -81,14 +85,14 @@ __device__ void build_merged_b(const GemmParams& p, int g, int n0, uint8_t* sBm,
     return v;
   };
 #pragma unroll 1
-  for (int i0 = w; i0 < BN; i0 += 8) {
+  for (int i0 = w; i0 < BN; i0 += 2 * kEpiWarps) {
     int plo[2], phi[2], nn[2], slot_lo[2];
     float lse[2][kPieces];
     uint4 v[2][kPieces][2];
     // issue every load of both rows (o_lat row, or up to kPieces partial pieces) first
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int i = i0 + 4 * r;
+      const int i = i0 + kEpiWarps * r;
       nn[r] = n0 + i;
       plo[r] = 0;
       phi[r] = -1;
@@ -121,7 +125,7 @@ __device__ void build_merged_b(const GemmParams& p, int g, int n0, uint8_t* sBm,
     }
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int i = i0 + 4 * r;
+      const int i = i0 + kEpiWarps * r;
       if (i >= BN) continue;
       uint4 out_lo = make_uint4(0, 0, 0, 0), out_hi = make_uint4(0, 0, 0, 0);
       if (nn[r] < p.N) {
@@ -313,10 +317,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 128);
+      mbar_init(&acc_empty[i], kEpiThreads);
     }
     mbar_init(drain, 1);
-    mbar_init(b_ready, 128);
+    mbar_init(b_ready, kEpiThreads);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -406,12 +410,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       umma_commit(drain);
     }
   } else {
-    // epilogue warps 2..5 → TMEM lane quadrant warp % 4
+    // epilogue warps 2 .. 1+kEpiWarps → TMEM lane quadrant warp % 4
     pdl_wait();   // outputs may be read by the kernel before this one
     const int quad = warp & 3;
     const int row = quad * 32 + static_cast<int>(lane_id());
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const int etid = static_cast<int>(threadIdx.x) - 64;   // 0..127
+    const int etid = static_cast<int>(threadIdx.x) - 64;   // 0 .. kEpiThreads-1
+    const int half = etid >> 7;   // the two warps of a lane quadrant split the 16-token blocks
     // the epilogue writes 16-byte vectors: every 8-row group must start 16-byte aligned (the C
     // ABI requires aligned outputs; a violation is reported, never written)
     const bool aligned_out =
@@ -436,10 +441,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!aligned_out) break;
       // 16-token blocks: lane = row, value i = token; bf16 into this warp's staging block as
       // [token][32 rows], then each lane writes two 16-byte pieces (8 rows of one token)
-      __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sEpi + (warp & 3) * 1024);
+      __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sEpi + (warp - 2) * 1024);
       const int mw = un.m0 + quad * 32;   // first row of this warp
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 16) {
+      for (int c0 = 16 * half; c0 < BN; c0 += 32) {
         if (un.n0 + c0 >= p.N) break;   // uniform across the warp
         float v[16];
         float2 cs[16];
