@@ -61,7 +61,8 @@ constexpr int gemm_smem_bytes() {
 // weights; merged rows are also written to o_lat (and their lse to lse_out).  The epilogue warps
 // (kEpiWarps) share the rows: warp w takes rows w, w+kEpiWarps, ... two at a time with all their
 // loads in flight (the merge is a chain of dependent steps per row, so more warps hide more);
-// lane l owns columns 16l .. 16l+15.  The tile's key prefix is read once (one value per lane).
+// lane l owns columns 16l .. 16l+15.  The tile's per-row piece records are read once (one per
+// lane) and handed around by shuffles.
 template <int BN>
 __device__ void build_merged_b(const GemmParams& p, int g, int n0, uint8_t* sBm, int etid) {
   const int w = etid >> 5, lane = etid & 31;
