@@ -87,14 +87,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
-// Arrive on a barrier in another CTA of the cluster (address from mapa), with release semantics
-// at cluster scope so this thread's earlier distributed-shared-memory stores are visible first.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                   remote_bar_addr)
-               : "memory");
-}
-
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -189,11 +181,6 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* s
                : "memory");
 }
 
-// Ask for `bytes` (multiple of 16) of contiguous global memory to be brought into L2.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ void tma_load_3d_hint(void* smem_dst, const CUtensorMap* m,
                                                  uint64_t* bar, int32_t c0, int32_t c1,
                                                  int32_t c2, uint64_t policy) {
@@ -208,12 +195,6 @@ __device__ __forceinline__ void tma_load_3d_hint(void* smem_dst, const CUtensorM
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 
@@ -292,7 +273,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
       : "memory");
 }
 
-
 // Raw 32-bit words to TMEM (16 columns) and wait for the store.
 __device__ __forceinline__ void tmem_st16_u32(uint32_t taddr, const uint32_t (&r)[16]) {
   __syncwarp();   // .sync.aligned: the whole warp, converged
@@ -302,16 +282,6 @@ __device__ __forceinline__ void tmem_st16_u32(uint32_t taddr, const uint32_t (&r
       "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-
-// 8 raw 32-bit words to TMEM and wait for the store.
-__device__ __forceinline__ void tmem_st8_u32(uint32_t taddr, const uint32_t (&r)[8]) {
-  __syncwarp();   // .sync.aligned: the whole warp, converged
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
 }
 
@@ -419,22 +389,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t ra
   return r;
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
-// Asynchronous 16-byte store into another CTA's shared memory; on arrival it performs
-// complete_tx(16) on the given mbarrier of that CTA (both addresses from mapa).
-__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, float a, float b, float c, float d,
-                                            uint32_t remote_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
-      ::"r"(remote_addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
-      : "memory");
-}
-
 // Arrive on a barrier of another CTA of the cluster without ordering earlier memory operations.
 // Callers that use it to release a buffer first consume every value they loaded from it (see
 // consume32), so the loads have completed before this instruction can issue.
@@ -464,11 +418,6 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 // Wait until every committed bulk copy of this thread has completed (destination written).
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-// Named barrier over `nthreads` threads (whole warps).
-__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Makes the 32 values "used" at this point in program order: the instructions producing them
