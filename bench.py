@@ -459,8 +459,10 @@ def run_reference(args) -> dict:
     res = None
     for _ in range(args.warmup):
         oracle_sample(w, inp, budget_s=0.0, max_rows=1)
+    # each step is a bounded sample; the whole run stays within about two minutes of oracle time
+    step_s = min(args.ref_step_seconds, max(0.5, 120.0 / max(1, args.steps)))
     for _ in range(args.steps):
-        res = oracle_sample(w, inp, budget_s=args.ref_step_seconds)
+        res = oracle_sample(w, inp, budget_s=step_s)
         per_step.append(res["value"])
     value = float(np.mean(per_step))
     return {
@@ -486,7 +488,9 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle CPU-baseline sample")
-    ap.add_argument("--ref-step-seconds", type=float, default=6.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=6.0,
+                    help="oracle time per step of --impl reference (capped so that all steps "
+                         "together take about two minutes)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time the eager C-ABI call instead of a CUDA-graph replay of it")
