@@ -43,3 +43,33 @@ def test_warmup_below_three_is_refused():
     r = subprocess.run(CMD[:6] + ["--warmup", "2"], capture_output=True, text=True, timeout=300,
                        cwd=ROOT)
     assert r.returncode != 0 and "--warmup must be >= 3" in r.stderr
+
+
+def test_algorithmic_work_matches_the_hand_count():
+    """The roofline's numerator: for the V3.2 decode batch (B=32, H=128, L=4096, each row sees
+    its 4097 keys) the attention must move every cached key once (512 latent + 64 rotary bf16 =
+    1152 B), read the absorbed query (128 padded heads x 576 bf16) and write o_lat (512 bf16 per
+    head); the flops are 2 per multiply-add of the score (576 wide) and P·V (512 wide) products."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    from mla_synth import make_inputs, workload
+    w = workload("v32_decode")
+    inp = make_inputs(w, seed=0)
+    work = bench.algorithmic_work(w, inp["start_pos"])
+    B, H, keys = 32, 128, 4097
+    assert work["keys"] == B * keys == 131104
+    assert work["cache_bytes"] == B * keys * 1152
+    assert work["attn_bytes"] == B * keys * 1152 + B * H * 576 * 2 + B * H * 512 * 2 == 159944704
+    assert work["attn_flops"] == 2 * B * keys * H * (576 + 512)
+    # whole step: weights (wq_b, wkv_b, fp32 gain), activations in/out, cache, output
+    weights = H * 192 * 1536 * 2 + H * 256 * 512 * 2 + 1536 * 4
+    assert work["weight_bytes"] == weights
+    assert work["bytes"] == 2 * B * 1536 * 2 + weights + B * keys * 1152 + B * H * 128 * 2
+    # a prefill chunk reads its sequence's cache prefix once, whatever the number of tokens
+    wp = workload("prefill_chunk")
+    inpp = make_inputs(wp, seed=0)
+    wk = bench.algorithmic_work(wp, inpp["start_pos"])
+    assert wk["cache_bytes"] == (2048 + 2048) * 1152
+    t = np.arange(2048)
+    assert wk["keys"] == int((2048 + t + 1).sum())
