@@ -37,7 +37,9 @@ Precision modes of ``decode`` / ``prefill``:
     [QH] mla-queries) and the absorbed q_nope (einsum of bf16 tensors, [AU] mla-decode).  Scores,
     softmax and everything after stay float64 (the fp32 softmax of the method).  This is the
     reference for the softmax probabilities, whose 1e-3 bound is tighter than the effect of those
-    four roundings.
+    four roundings.  Pinned by a pure-Python scalar enumeration with its own bit-level bf16
+    rounding, compared bit for bit on inputs whose sums are exact, and by mutations that drop
+    each rounding in turn.
 """
 from __future__ import annotations
 

@@ -8,7 +8,7 @@ import pytest
 
 import oracle
 import oracle.mla_oracle as om
-from test_oracle_pins import _brute_decode_one
+from test_oracle_pins import _brute_decode_one, bf16_mode_mismatches
 
 
 def _max_err_vs_brute(seed=0):
@@ -72,3 +72,34 @@ def test_planted_mistake_is_caught(monkeypatch, name, target, replacement):
     assert _max_err_vs_brute() < 1e-12
     monkeypatch.setattr(om, target, replacement)
     assert _max_err_vs_brute() > 1e-6, name
+
+
+# ------------------------------------------------------------------------------------------
+# Placement of the bf16 roundings in query_precision="bf16"
+# ------------------------------------------------------------------------------------------
+_ROUNDING_POINTS = ["RMSNorm output", "wq_b output (before RoPE)", "q_pe after RoPE",
+                    "absorbed q_nope"]
+
+
+@pytest.mark.parametrize("skip", range(4), ids=_ROUNDING_POINTS)
+def test_dropped_bf16_rounding_is_caught(monkeypatch, skip):
+    """Drop one of the four roundings (the oracle rounds in that order on every call); dropping
+    the one after RoPE is the "round q_pe before RoPE instead of after" slip."""
+    assert bf16_mode_mismatches(0)[0] == 0
+    real = om.round_bf16
+    calls = {"n": 0}
+
+    def dropped(a):
+        k = calls["n"]
+        calls["n"] += 1
+        return np.asarray(a, np.float64) if k % 4 == skip else real(a)
+
+    monkeypatch.setattr(om, "round_bf16", dropped)
+    bad = sum(bf16_mode_mismatches(s)[0] for s in range(3))
+    assert bad > 0, _ROUNDING_POINTS[skip]
+
+
+def test_wrong_rounding_format_is_caught(monkeypatch):
+    monkeypatch.setattr(om, "round_bf16",
+                        lambda a: np.asarray(a, np.float64).astype(np.float16).astype(np.float64))
+    assert bf16_mode_mismatches(0)[0] > 0

@@ -9,6 +9,7 @@ import cmath
 import json
 import math
 import os
+import struct
 
 import numpy as np
 import pytest
@@ -271,25 +272,49 @@ def test_zero_query_averages_latents():
 # ------------------------------------------------------------------------------------------
 # Brute force on tiny inputs (pure-Python scalar loops written from the pages' description)
 # ------------------------------------------------------------------------------------------
-def _brute_decode_one(x, gamma, wq_b, wkv_b, cache, pos, H, C, Dn, Dr, Dv, theta, eps):
+def _bf16_bits(v: float) -> float:
+    """Nearest bfloat16 value to the float64 ``v`` (ties to even), found by editing the IEEE-754
+    bit pattern: keep the sign, the exponent and the top 7 of the 52 stored mantissa bits."""
+    (u,) = struct.unpack("<Q", struct.pack("<d", v))
+    drop = 52 - 7
+    half = 1 << (drop - 1)
+    keep_lsb = (u >> drop) & 1
+    u = (u + half - 1 + keep_lsb) & ~((1 << drop) - 1)   # a carry may bump the exponent: correct
+    (r,) = struct.unpack("<d", struct.pack("<Q", u))
+    return r
+
+
+def _brute_decode_one(x, gamma, wq_b, wkv_b, cache, pos, H, C, Dn, Dr, Dv, theta, eps,
+                      rnd=None, trace=None):
+    """Scalar enumeration of one decode row.  ``rnd`` (optional) rounds the query side where the
+    pages' tensors are bf16: the RMSNorm output, the wq_b output, the rotated q_pe and the absorbed
+    q_nope.  ``trace`` (a dict) receives those four query tensors."""
+    keep = rnd if rnd is not None else (lambda v: v)
     R = len(x)
     ms = sum(v * v for v in x) / R
-    y = [gamma[j] * x[j] / math.sqrt(ms + eps) for j in range(R)]
+    y = [keep(gamma[j] * (x[j] / math.sqrt(ms + eps))) for j in range(R)]
     scale = (Dn + Dr) ** -0.5
     outs, lses = [], []
+    if trace is not None:
+        trace.update(y=y, q_nope=[], q_pe=[], q_lat=[])
     for h in range(H):
-        qh = [sum(y[k] * wq_b[h * (Dn + Dr) + j][k] for k in range(R)) for j in range(Dn + Dr)]
+        qh = [keep(sum(y[k] * wq_b[h * (Dn + Dr) + j][k] for k in range(R))) for j in range(Dn + Dr)]
         q_nope, q_pe = qh[:Dn], qh[Dn:]
         q_rot = []
         for i in range(Dr // 2):
             z = complex(q_pe[2 * i], q_pe[2 * i + 1]) * cmath.exp(1j * pos * theta ** (-2 * i / Dr))
-            q_rot += [z.real, z.imag]
+            q_rot += [keep(z.real), keep(z.imag)]
+        q_lat = [keep(sum(q_nope[dd] * wkv_b[h * (Dn + Dv) + dd][c] for dd in range(Dn)))
+                 for c in range(C)]
+        if trace is not None:
+            trace["q_nope"].append(q_nope)
+            trace["q_pe"].append(q_rot)
+            trace["q_lat"].append(q_lat)
         logits = []
         for t in range(pos + 1):
             acc = 0.0
             for c in range(C):
-                w_uk_col = sum(q_nope[dd] * wkv_b[h * (Dn + Dv) + dd][c] for dd in range(Dn))
-                acc += w_uk_col * cache[t][c]
+                acc += q_lat[c] * cache[t][c]
             acc += sum(q_rot[r] * cache[t][C + r] for r in range(Dr))
             logits.append(acc * scale)
         mx = max(logits)
@@ -338,6 +363,78 @@ def test_round_bf16_matches_torch_and_ties_to_even():
     assert oracle.round_bf16(np.array(1 + 2.0 ** -8 + 2.0 ** -40)) == 1 + 2.0 ** -7
     x = rng.standard_normal(1000)
     np.testing.assert_array_equal(oracle.round_bf16(oracle.round_bf16(x)), oracle.round_bf16(x))
+
+
+def test_bf16_rounding_by_bits_matches_torch():
+    """The enumeration's own bf16 rounding (bit editing) against torch's float32 -> bfloat16."""
+    import torch
+    rng = np.random.default_rng(15)
+    a = (rng.standard_normal(20000) * np.exp(rng.uniform(-30, 30, 20000))).astype(np.float32)
+    ref = torch.from_numpy(a).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(np.array([_bf16_bits(float(v)) for v in a]), ref)
+    assert _bf16_bits(1 + 2.0 ** -8) == 1.0                 # tie, even neighbour below
+    assert _bf16_bits(1 + 3 * 2.0 ** -8) == 1 + 2.0 ** -6   # tie, even neighbour above
+    assert _bf16_bits(-(1 + 2.0 ** -8 + 2.0 ** -40)) == -(1 + 2.0 ** -7)
+    assert _bf16_bits(2 - 2.0 ** -9) == 2.0                 # carry into the exponent
+
+
+def _dyadic_setup(seed, L=5):
+    """Small-integer / dyadic inputs: every sum of products the query side forms is exact in
+    float64, so the only inexact steps are the RMSNorm square root and the RoPE angles, and the
+    bf16 roundings can be compared bit for bit."""
+    rng = np.random.default_rng(300 + seed)
+    H, R, C, Dn, Dr, Dv = 2, 8, 4, 2, 4, 2
+    x = rng.integers(-3, 4, (2, R)).astype(float)
+    x[np.all(x == 0, axis=1), 0] = 1.0
+    return dict(
+        x=x, gamma=rng.integers(1, 4, R) / 2.0,
+        wq_b=rng.integers(-3, 4, (H * (Dn + Dr), R)) / 8.0,
+        wkv_b=rng.integers(-3, 4, (H * (Dn + Dv), C)) / 4.0,
+        cache=rng.integers(-3, 4, (2, L, C + Dr)).astype(float),
+        pos=np.array([L - 1, 2]), dims=dict(H=H, C=C, Dn=Dn, Dr=Dr, Dv=Dv))
+
+
+def bf16_mode_mismatches(seed):
+    """Oracle decode in query_precision="bf16" against the rounded scalar enumeration: the number
+    of query elements (y, q_nope, q_pe, q_lat) that differ bit for bit, and the largest output /
+    lse difference."""
+    S = _dyadic_setup(seed)
+    d = S["dims"]
+    r = oracle.decode(S["x"], S["gamma"], S["wq_b"], S["wkv_b"], S["cache"], S["pos"],
+                      n_heads=d["H"], kv_lora=d["C"], nope=d["Dn"], rope=d["Dr"], v=d["Dv"],
+                      want_intermediates=True, query_precision="bf16")
+    bad, err = 0, 0.0
+    for b in range(2):
+        tr = {}
+        o, l = _brute_decode_one(list(S["x"][b]), list(S["gamma"]), S["wq_b"].tolist(),
+                                 S["wkv_b"].tolist(), S["cache"][b].tolist(), int(S["pos"][b]),
+                                 d["H"], d["C"], d["Dn"], d["Dr"], d["Dv"], 10000.0, 1e-6,
+                                 rnd=_bf16_bits, trace=tr)
+        for k in ("y", "q_nope", "q_pe", "q_lat"):
+            bad += int(np.sum(np.asarray(r[k][b]) != np.asarray(tr[k])))
+        err = max(err, float(np.max(np.abs(r["out"][b] - np.array(o)))),
+                  float(np.max(np.abs(r["lse"][b] - np.array(l)))))
+    return bad, err
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_bf16_query_mode_matches_rounded_enumeration(seed):
+    """query_precision="bf16" rounds exactly where the pages' tensors are bf16: RMSNorm output
+    ("Attention update" rmsnorm: ``.to(dtype)``), the wq_b Linear output and the rotated q_pe
+    ("Query heads" mla-queries), the absorbed q_nope ("Attention update" mla-decode einsum)."""
+    bad, err = bf16_mode_mismatches(seed)
+    assert bad == 0
+    assert err < 1e-12
+    # the roundings are active on these inputs: the exact mode differs
+    S = _dyadic_setup(seed)
+    d = S["dims"]
+    kw = dict(n_heads=d["H"], kv_lora=d["C"], nope=d["Dn"], rope=d["Dr"], v=d["Dv"],
+              want_intermediates=True)
+    ex = oracle.decode(S["x"], S["gamma"], S["wq_b"], S["wkv_b"], S["cache"], S["pos"], **kw)
+    bq = oracle.decode(S["x"], S["gamma"], S["wq_b"], S["wkv_b"], S["cache"], S["pos"],
+                       query_precision="bf16", **kw)
+    for k in ("y", "q_nope", "q_pe", "q_lat"):
+        assert not np.array_equal(ex[k], bq[k]), k
 
 
 def test_bf16_query_mode_stays_close_to_exact():
