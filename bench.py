@@ -1,16 +1,22 @@
 """Benchmark of the absorbed-MLA hot path on B200.
 
-One step = one full decode call (q_norm → wq_b+RoPE → W_UK absorption → latent attention over
-the cache → combine → W_UV) for the DeepSeek-V3.2-shaped decode batch: B=32 sequences, H=128,
-cache L=4096 (keys 0..4096), bf16, synthetic seeded inputs resident in HBM.  Between timed steps
-L2 is flushed by writing a 256 MiB buffer and then reading another 256 MiB buffer (both untimed):
-the step starts with none of its data in L2, and without 126 MB of dirty flush lines that the
-step's own loads and stores would otherwise have to write back (the step's inputs are 261 MB).
-The timed steps replay a CUDA graph of one call on a dedicated stream (--no-graph: the eager
-call); the stage breakdown and the end-to-end number use eager calls through the C ABI.
+One step = one full call of the path (q_norm → wq_b+RoPE → W_UK absorption → latent attention over
+the cache → split merge → W_UV) on synthetic seeded inputs resident in HBM.  The default run times
+every configuration of the method in turn:
+  ragged_decode  B=64, H=128, cache lengths L_b ~ U{1024..32768}, residual RMSNorm  (headline:
+                 the largest single-GPU configuration; top-level value / config)
+  tiny_decode    B=2,  H=16,  L=128
+  v32_decode     B=32, H=128, L=4096
+  prefill_chunk  B=1,  T=2048 new tokens after 2048 cached, H=128 (causal), reported in TFLOP/s
+  kimi_decode    B=128, H=64, L=2048
+and prints ONE JSON line: the headline's numbers at top level and the others under "workloads".
+Between timed steps L2 is flushed by writing a 256 MiB buffer and then reading another 256 MiB
+buffer (both untimed): every step starts with none of its data in L2.  The timed steps replay a
+CUDA graph of one C-ABI call on a dedicated stream (--no-graph: the eager call); the per-kernel
+breakdown (roofline) and the end-to-end number use eager calls through the C ABI.
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-        [--workload v32_decode|kimi_decode|ragged_decode|tiny_decode|prefill_chunk]
+        [--workload all|ragged_decode|tiny_decode|v32_decode|prefill_chunk|kimi_decode]
 For N > 1 launch one process per GPU with torch.distributed.run; every rank runs its own replica
 batch (the path shards by sequence with no exchange: weak scaling) and rank 0 prints one JSON line.
 """
@@ -35,6 +41,8 @@ from mla_synth import keys_per_row, make_inputs, workload  # noqa: E402
 
 METRIC = "MLA decode queries/s + HBM GB/s (% peak); prefill-chunk TFLOP/s (% peak)"
 FLUSH_BYTES = 256 << 20
+HEADLINE = "ragged_decode"
+WORKLOAD_ORDER = ("ragged_decode", "tiny_decode", "v32_decode", "prefill_chunk", "kimi_decode")
 
 
 # ------------------------------------------------------------------------------------------
@@ -55,7 +63,9 @@ def algorithmic_work(w, start_pos: np.ndarray) -> dict:
     out = rows * H * Dv * 2
     flops = (2 * rows * R * H * (Dn + Dr) + 2 * rows * H * Dn * C
              + 2 * int(keys.sum()) * H * ((C + Dr) + C) + 2 * rows * H * C * Dv)
-    attn_bytes = cache + rows * H * (C + Dr) * 2 + rows * H * C * 2
+    # the attention kernel's roofline counts only what the method must move: every cache row a
+    # query attends crosses HBM once (the absorbed query and o_lat are intermediates of this build)
+    attn_bytes = cache
     attn_flops = 2 * int(keys.sum()) * H * ((C + Dr) + C)
     return dict(bytes=act + weights + cache + out, flops=flops, cache_bytes=cache,
                 weight_bytes=weights, attn_bytes=attn_bytes, attn_flops=attn_flops,
@@ -219,18 +229,18 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------
 # Our arm
 # ------------------------------------------------------------------------------------------
-def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
+def run_workload(name: str, args, rank: int, world: int, local_rank: int) -> dict | None:
+    """Times one configuration on this rank's GPU; returns its JSON entry on rank 0 (None on the
+    other ranks).  Every rank takes the same collective steps (two barriers, one all-reduce)."""
     import torch
     import torch.distributed as dist
 
-    torch.cuda.set_device(local_rank)
     dev = f"cuda:{local_rank}"
-    from head_latent_attention_11_b200 import (build, mla_enable_stage_timing,
-                                               mla_last_launch_count, mla_stage_times)
-    build.build()
+    from head_latent_attention_11_b200 import (mla_enable_stage_timing, mla_last_launch_count,
+                                               mla_stage_times)
     from head_latent_attention_11_b200.runtime import MLARuntime
 
-    w = workload(args.workload)
+    w = workload(name)
     inp = make_inputs(w, seed=args.seed + rank)
     work = algorithmic_work(w, inp["start_pos"])
     B, T, H = w.batch, w.tokens, w.dims.n_heads
@@ -254,9 +264,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     out = torch.empty(out_shape, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    # a dedicated stream (the legacy default stream serialises with every other stream and
-    # measured ~6 µs slower per step); torch's flush kernels run on it too
+    # a dedicated stream (the legacy default stream serialises with every other stream); torch's
+    # flush kernels run on it too
     stream = torch.cuda.Stream(device=dev)
+    prev_stream = torch.cuda.current_stream(dev)
     torch.cuda.set_stream(stream)
 
     def flush_l2(i: int) -> None:
@@ -274,10 +285,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         step()
     torch.cuda.synchronize()
     if rt.sync_status(stream) != 0:
-        raise RuntimeError("device status set during warm-up")
-    # The timed steps replay a CUDA graph of one step (the same six kernels with the same
-    # arguments, chained by programmatic dependent launch, without per-call host work); --no-graph
-    # times the eager C-ABI call instead.
+        raise RuntimeError(f"{name}: device status set during warm-up")
     graph = None
     if not args.no_graph:
         graph = torch.cuda.CUDAGraph()
@@ -286,7 +294,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         graph.replay()
         torch.cuda.synchronize()
         if rt.sync_status(stream) != 0:
-            raise RuntimeError("device status set by the captured step")
+            raise RuntimeError(f"{name}: device status set by the captured step")
     run_step = graph.replay if graph is not None else step
 
     # ---- timed region: K steps, L2 flushed before each (flush not timed)
@@ -295,11 +303,11 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     clocks = ClockSampler(local_rank)
     clocks.start()
     # keep the GPU busy for ~0.5 s right before the timed steps (same flush + step, untimed) so
-    # that the clock record holds enough samples taken under this load
+    # that the clock record holds samples taken under this load
     clocks.mark("load")
     t_load = time.perf_counter()
     while time.perf_counter() - t_load < 0.5:
-        for i in range(32):
+        for i in range(16):
             flush_l2(i)
             run_step()
         torch.cuda.synchronize()
@@ -319,18 +327,18 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     clk = clocks.stop()
     launches = mla_last_launch_count(rt.ctx)
     if rt.sync_status(stream) != 0:
-        raise RuntimeError("device status set during the timed steps")
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = float(sum(step_ms))
+        raise RuntimeError(f"{name}: device status set during the timed steps")
+    total_ms = float(sum(s.elapsed_time(e) for s, e in zip(starts, ends)))
 
-    # ---- stage breakdown (separate pass with per-kernel events; not part of `value`)
+    # ---- per-kernel breakdown: a separate pass of eager calls on the same stream with CUDA
+    # events around every kernel (not part of `value`)
     mla_enable_stage_timing(rt.ctx, True)
     stage_acc: dict[str, list[float]] = {}
     for i in range(max(3, min(args.steps, 20))):
         flush_l2(i)
         step()
-        for name, ms in mla_stage_times(rt.ctx):
-            stage_acc.setdefault(name, []).append(ms)
+        for kname, ms in mla_stage_times(rt.ctx):
+            stage_acc.setdefault(kname, []).append(ms)
     mla_enable_stage_timing(rt.ctx, False)
     stages = {k: float(np.mean(v)) for k, v in stage_acc.items()}
 
@@ -363,16 +371,19 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     # ---- max over ranks
     total_ms, e2e_total = max_over_ranks([total_ms, float(np.sum(e2e_ms))], device=dev)
     rt.close()
+    torch.cuda.set_stream(prev_stream)
+    del graph, rt, cache, wq_b, wkv_b, flush, flush_rd
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
     if rank != 0:
         return None
 
     peaks = measured_peaks()
     ms_per_step = total_ms / args.steps
-    units = B * T
     if w.mode == "decode":
-        value = aggregate_throughput(units, args.steps, world, total_ms)
+        value = aggregate_throughput(B * T, args.steps, world, total_ms)
         unit = "queries/s"
-        e2e_value = aggregate_throughput(units, args.steps, world, e2e_total)
+        e2e_value = aggregate_throughput(B * T, args.steps, world, e2e_total)
     else:
         value = world * work["flops"] * args.steps / (total_ms / 1e3) / 1e12
         unit = "TFLOP/s"
@@ -384,44 +395,47 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": profiled_traffic(w.name), "kernel": "latent_attention",
                 "algorithmic_bytes_per_launch": work["attn_bytes"],
+                "algorithmic_bytes_rule": "cache rows attended x 1152 B (576 bf16)",
+                "kernel_ms": round(attn_ms, 5),
                 "peak_source": peaks["source"] + " (hbm_gbs, copy burst)"}
     else:
         achieved = work["attn_flops"] / (attn_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1),
-                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops_sustained"], 4), "traffic": None,
-                "kernel": "latent_attention", "algorithmic_flops_per_launch": work["attn_flops"],
-                "peak_source": peaks["source"] + " (bf16_tflops_sustained)"}
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "traffic": profiled_traffic(w.name), "kernel": "latent_attention",
+                "algorithmic_flops_per_launch": work["attn_flops"],
+                "algorithmic_flops_rule": "2 x visible (query, key) pairs x H x (576 + 512)",
+                "kernel_ms": round(attn_ms, 5),
+                "peak_source": peaks["source"] + " (bf16_tflops, burst: a kernel of a few ms)"}
     step_gbs = work["bytes"] / (ms_per_step / 1e3) / 1e9
-    line = {
-        "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) latents/caches, N(0,1/fan_in) weights)",
+    return {
+        "value": round(value, 2), "unit": unit, "ms_per_step": round(ms_per_step, 5),
         "config": {"workload": w.name, "batch": B, "tokens": T, "n_heads": H,
                    "cache_keys_per_step": work["keys"], "q_lora": 1536, "kv_lora": 512,
-                   "rope": 64, "v": 128,
+                   "rope": 64, "v": 128, "residual": bool(w.residual),
                    "l2": "flushed before every timed step: 256 MiB write, then 256 MiB read of another buffer (untimed)",
                    "launch": "eager C-ABI call" if args.no_graph else "CUDA graph of one C-ABI call, replayed on a dedicated stream",
                    "parallelism": f"replicas x{world} (sequence-sharded, no collective)"},
         "hbm": {"step_bytes": work["bytes"], "step_gbs": round(step_gbs, 1),
                 "frac_of_peak": round(step_gbs / peaks["hbm_gbs"], 4)},
         "tflops_step": round(work["flops"] / (ms_per_step / 1e3) / 1e12, 2),
+        "tensor_frac_of_peak": round(work["flops"] / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
         "roofline": roof,
         "stages_ms": {k: round(v, 5) for k, v in stages.items()},
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 2), "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_total / args.steps, 5)},
         "gpu_launches": launches * args.steps,
+        "kernels_per_step": launches,
     }
-    return line
 
 
 # ------------------------------------------------------------------------------------------
 # CPU legs: the fp64 oracle on the host cores (bounded sample)
 # ------------------------------------------------------------------------------------------
 def oracle_sample(w, inp, budget_s: float, max_rows: int | None = None) -> dict:
-    """Run the oracle on sequences 0, 1, ... until ~budget_s of CPU time; returns rate."""
+    """Run the oracle on query rows 0, 1, ... (cycling over the batch) until ~budget_s of CPU
+    time; returns the rate in the workload's unit."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from mla_cases import oracle_decode, oracle_prefill
     try:
@@ -438,7 +452,8 @@ def oracle_sample(w, inp, budget_s: float, max_rows: int | None = None) -> dict:
                 break
         el = time.perf_counter() - t0
         return dict(value=done / el, unit="queries/s", cores=cores,
-                    sample=f"{done} of the {w.batch} sequences' decode (all {w.dims.n_heads} heads) in {el:.1f} s")
+                    sample=f"{done} decode rows (cycling over the {w.batch} sequences, all "
+                           f"{w.dims.n_heads} heads) in {el:.1f} s")
     T = w.tokens
     work = algorithmic_work(w, inp["start_pos"])
     per_token = work["flops"] / T
@@ -449,11 +464,13 @@ def oracle_sample(w, inp, budget_s: float, max_rows: int | None = None) -> dict:
             break
     el = time.perf_counter() - t0
     return dict(value=done * per_token / el / 1e12, unit="TFLOP/s", cores=cores,
-                sample=f"{done} of the {T} chunk tokens in {el:.1f} s")
+                sample=f"{done} chunk tokens (of {T}, all {w.dims.n_heads} heads; flops "
+                       f"credited at the chunk's mean per token) in {el:.1f} s")
 
 
 def run_reference(args) -> dict:
-    w = workload(args.workload)
+    name = HEADLINE if args.workload == "all" else args.workload
+    w = workload(name)
     inp = make_inputs(w, seed=args.seed)
     per_step = []
     res = None
@@ -484,10 +501,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="v32_decode")
+    ap.add_argument("--workload", default="all", choices=("all",) + WORKLOAD_ORDER)
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0,
-                    help="budget of the oracle CPU-baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="budget of each workload's oracle CPU-baseline sample")
     ap.add_argument("--ref-step-seconds", type=float, default=6.0,
                     help="oracle time per step of --impl reference (capped so that all steps "
                          "together take about two minutes)")
@@ -507,20 +524,40 @@ def main(argv=None):
             print(json.dumps(run_reference(args)), flush=True)
         return 0
 
+    import torch
+    torch.cuda.set_device(local_rank)
     if world > 1:
         import datetime
-        import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    line = run_ours(args, rank, world, local_rank)
-    if line is not None:
-        if not args.no_cpu_baseline:
-            w = workload(args.workload)
-            inp = make_inputs(w, seed=args.seed)
-            cb = oracle_sample(w, inp, budget_s=args.cpu_seconds)
-            line["cpu_baseline"] = {"value": round(cb["value"], 4), "unit": cb["unit"],
-                                    "cores": cb["cores"], "kind": "oracle", "sample": cb["sample"]}
+    from head_latent_attention_11_b200 import build
+    build.build()
+
+    names = WORKLOAD_ORDER if args.workload == "all" else (args.workload,)
+    entries = {n: run_workload(n, args, rank, world, local_rank) for n in names}
+    if rank == 0:
+        head_name = names[0]
+        head = entries[head_name]
+        if not args.no_cpu_baseline and world == 1:
+            for n in names:
+                w = workload(n)
+                cb = oracle_sample(w, make_inputs(w, seed=args.seed), budget_s=args.cpu_seconds)
+                entries[n]["cpu_baseline"] = {"value": round(cb["value"], 4), "unit": cb["unit"],
+                                              "cores": cb["cores"], "kind": "oracle",
+                                              "sample": cb["sample"]}
+        line = {
+            "metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) latents/caches/residual, N(0,1/fan_in) weights, "
+                    "U(0.5,1.5) gain)",
+        }
+        line.update({k: v for k, v in head.items() if k not in ("value", "unit", "ms_per_step")})
+        line["gpu_launches"] = sum(e["gpu_launches"] for e in entries.values())
+        line["gpu_launches_note"] = ("kernels of this library launched in the timed steps of "
+                                     "every workload below (headline included)")
+        if len(names) > 1:
+            line["workloads"] = {n: entries[n] for n in names[1:]}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -22,7 +22,6 @@ using namespace mla;
 
 namespace {
 
-constexpr int kMinKeysPerPair = 256;
 constexpr int kMaxStages = 8;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -199,15 +198,6 @@ mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_E
     cudaError_t _e = (expr);                        \
     if (_e != cudaSuccess) return MLA_ERR_CUDA;     \
   } while (0)
-
-bool cache_args_ok(const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe, int64_t pe_sb,
-                   int64_t pe_st) {
-  if (!kv || !pe || !aligned(kv, 16) || !aligned(pe, 16)) return false;
-  if (kv_st < kC || pe_st < kDr || kv_sb < 1 || pe_sb < 1) return false;
-  if ((kv_st * 2) % 16 || (pe_st * 2) % 16 || (kv_sb * 2) % 16 || (pe_sb * 2) % 16) return false;
-  if (kv_st * 2 >= (1ll << 40) || kv_sb * 2 >= (1ll << 40) || pe_sb * 2 >= (1ll << 40)) return false;
-  return true;
-}
 
 // The whole path for `rows` query rows.  decode: start_pos_dev != null, T = 1.
 mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int32_t* start_pos_dev,

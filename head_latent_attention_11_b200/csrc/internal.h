@@ -171,6 +171,24 @@ cudaError_t launch_transpose_uk(const bf16* wkv_b, bf16* w_ukt, int n_heads, cud
 cudaError_t gemm_prepare();        // one-time per-device attribute set-up
 cudaError_t attention_prepare();
 
+// Smallest key range the attention kernel gives one SM pair (split-K granularity).
+constexpr int kMinKeysPerPair = 256;
+
+// Host-side check of the cache arguments shared by every entry point that reads the cache:
+// non-null, 16-byte aligned bases, rows at least C (kv) / Dr (pe) wide, row and batch strides
+// multiples of 16 bytes and below 2^40 bytes (tensor-map limits).  Strides in elements.
+inline bool cache_args_ok(const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,
+                          int64_t pe_sb, int64_t pe_st) {
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!kv || !pe || !al16(kv) || !al16(pe)) return false;
+  if (kv_st < kC || pe_st < kDr || kv_sb < 1 || pe_sb < 1) return false;
+  if ((kv_st * 2) % 16 || (pe_st * 2) % 16 || (kv_sb * 2) % 16 || (pe_sb * 2) % 16) return false;
+  if (kv_st * 2 >= (1ll << 40) || pe_st * 2 >= (1ll << 40) || kv_sb * 2 >= (1ll << 40) ||
+      pe_sb * 2 >= (1ll << 40))
+    return false;
+  return true;
+}
+
 // Token-tile width the GEMM launcher picks for N token rows (the B operand's TMA box height).
 inline int gemm_bn(int n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : 256; }
 

@@ -6,8 +6,9 @@
 // serves them: the caller passes its inputs and outputs, and the only other device memory used
 // is the fixed scratch array below, part of the library's image on every device that loads it.
 //
-// The scratch holds the per-row key prefix, the split-K partial outputs of at most
-// kNoAllocPairs SM pairs and a status word.  Limits: rows <= kNoAllocMaxRows; the attention
+// The scratch holds the per-row key prefix, the first row of each SM pair's key range, the
+// per-row piece records and the split-K partial outputs of at most kNoAllocPairs SM pairs; the
+// caller's status word receives device-side errors.  Limits: rows <= kNoAllocMaxRows; the attention
 // splits over at most kNoAllocPairs pairs (fewer SMs than the context path on large GPUs).
 //
 // Set-up: the first call on a device (with that device current) resolves the array's device
@@ -15,6 +16,8 @@
 // make that first call before capturing the stream into a CUDA graph.  Every call shares the
 // same array, so calls that may overlap on the GPU (different streams, different threads)
 // race on it and must be serialised by the caller.
+#include <math.h>
+
 #include <mutex>
 
 #include "mla.h"
@@ -26,8 +29,7 @@ namespace {
 
 constexpr int kNoAllocMaxRows = 4096;
 constexpr int kNoAllocPairs = 16;
-constexpr size_t kOffStatus = 0;
-constexpr size_t kOffPrefix = 256;
+constexpr size_t kOffPrefix = 0;
 constexpr size_t kOffPartO = kOffPrefix + ((static_cast<size_t>(kNoAllocMaxRows) + 1) * 8 + 255) / 256 * 256;
 constexpr size_t kOffPartLse = kOffPartO + static_cast<size_t>(kNoAllocPairs) * 2 * 128 * kC * 2;
 constexpr size_t kOffPairRow = kOffPartLse + static_cast<size_t>(kNoAllocPairs) * 2 * 128 * 4;
@@ -56,17 +58,17 @@ extern "C" mla_status mla_latent_attention_noalloc(
     float softmax_scale, const void* kv_cache, int64_t kv_stride_b, int64_t kv_stride_t,
     const void* pe_cache, int64_t pe_stride_b, int64_t pe_stride_t, int32_t max_seq_len,
     void* o_lat, float* lse, int32_t* status, cudaStream_t stream) {
-  if (!q_abs || !start_pos || !kv_cache || !pe_cache || !o_lat) return MLA_ERR_INVALID_ARG;
+  if (!q_abs || !start_pos || !o_lat || !status) return MLA_ERR_INVALID_ARG;
   if (rows < 1 || rows > kNoAllocMaxRows) return MLA_ERR_INVALID_ARG;   // beyond the scratch
   if (n_heads < 16 || n_heads > 128 || n_heads % 16 != 0) return MLA_ERR_UNSUPPORTED;
-  if (max_seq_len < 64 || !(softmax_scale > 0.f)) return MLA_ERR_INVALID_ARG;
-  if (!aligned16(q_abs) || !aligned16(o_lat) || !aligned16(kv_cache) || !aligned16(pe_cache) ||
-      (reinterpret_cast<uintptr_t>(start_pos) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
-      (status && (reinterpret_cast<uintptr_t>(status) & 3u)))
+  if (max_seq_len < 64 || max_seq_len > (1 << 24) || !(softmax_scale > 0.f) ||
+      !isfinite(softmax_scale))
     return MLA_ERR_INVALID_ARG;
-  if (kv_stride_t < kC || pe_stride_t < kDr || kv_stride_b < 1 || pe_stride_b < 1 ||
-      (kv_stride_t * 2) % 16 || (pe_stride_t * 2) % 16 || (kv_stride_b * 2) % 16 ||
-      (pe_stride_b * 2) % 16)
+  if (!aligned16(q_abs) || !aligned16(o_lat) || (reinterpret_cast<uintptr_t>(start_pos) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+      (reinterpret_cast<uintptr_t>(status) & 3u))
+    return MLA_ERR_INVALID_ARG;
+  if (!cache_args_ok(kv_cache, kv_stride_b, kv_stride_t, pe_cache, pe_stride_b, pe_stride_t))
     return MLA_ERR_INVALID_ARG;
 
   int dev = 0;
@@ -84,7 +86,7 @@ extern "C" mla_status mla_latent_attention_noalloc(
     }
     scratch = su.scratch;
   }
-  int* st = status ? status : reinterpret_cast<int*>(scratch + kOffStatus);
+  int* st = status;
   long long* prefix = reinterpret_cast<long long*>(scratch + kOffPrefix);
   __half* part_o = reinterpret_cast<__half*>(scratch + kOffPartO);
   float* part_lse = reinterpret_cast<float*>(scratch + kOffPartLse);
@@ -97,10 +99,8 @@ extern "C" mla_status mla_latent_attention_noalloc(
                            pe_stride_t, rows, max_seq_len, q_abs, rows, o_lat, n_heads, part_o, pairs))
     return MLA_ERR_INVALID_ARG;
 
-  // the internal status word starts at zero on every call; the prefix and partials are
-  // written before they are read within the call
-  if (!status && cudaMemsetAsync(st, 0, sizeof(int), stream) != cudaSuccess) return MLA_ERR_CUDA;
-
+  // the prefix and partials in the scratch array are written before they are read within the
+  // call; nothing in it needs clearing
   RmsParams rp{};
   rp.rows = rows;
   rp.T = 1;
@@ -110,7 +110,7 @@ extern "C" mla_status mla_latent_attention_noalloc(
   rp.pair_row = pair_row;
   rp.row_pieces = row_pieces;
   rp.n_pairs = pairs;
-  rp.min_keys_per_pair = 256;
+  rp.min_keys_per_pair = kMinKeysPerPair;
   rp.status = st;
   if (launch_key_prefix(rp, stream) != cudaSuccess) return MLA_ERR_CUDA;
 
@@ -122,7 +122,7 @@ extern "C" mla_status mla_latent_attention_noalloc(
   ap.n_heads = n_heads;
   ap.scale = softmax_scale;
   ap.scale_log2 = softmax_scale * 1.4426950408889634f;
-  ap.min_keys_per_pair = 256;
+  ap.min_keys_per_pair = kMinKeysPerPair;
   ap.o_lat = static_cast<bf16*>(o_lat);
   ap.lse_out = lse;
   ap.max_seq_len = max_seq_len;
@@ -137,7 +137,7 @@ extern "C" mla_status mla_latent_attention_noalloc(
   cp.rows = rows;
   cp.n_heads = n_heads;
   cp.n_pairs = pairs;
-  cp.min_keys_per_pair = 256;
+  cp.min_keys_per_pair = kMinKeysPerPair;
   cp.part_o = part_o;
   cp.part_lse = part_lse;
   cp.row_pieces = row_pieces;

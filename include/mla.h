@@ -117,7 +117,11 @@ mla_status mla_rmsnorm(const void* x, void* residual, const float* gain, int32_t
  *   out [B, H, Dv] bf16;  lse [B, H] fp32 or NULL — natural-log sum of exp(scaled scores);
  *   logits [B, H, max_seq_len] fp32 or NULL — debug copy of the scaled scores s (only keys
  *     0..start_pos[b] are written).
- * 1 <= B <= cfg.max_rows. */
+ * 1 <= B <= cfg.max_rows.
+ * Range: a row whose keys are split between SM pairs keeps each piece's normalised partial output
+ * (a convex combination of cached latents) in fp16 before the log-sum-exp merge, so cached latent
+ * values must lie within fp16's range (|value| <= 65504); larger values overflow to inf in those
+ * rows only.  The same holds for mla_prefill_chunk. */
 mla_status mla_decode(mla_ctx* ctx, const void* q_latent, void* residual, const int32_t* start_pos,
                       const void* kv_cache, int64_t kv_stride_b, int64_t kv_stride_t,
                       const void* pe_cache, int64_t pe_stride_b, int64_t pe_stride_t, int32_t B,
@@ -146,8 +150,12 @@ mla_status mla_prefill_chunk(mla_ctx* ctx, const void* q_latent, void* residual,
  *   caches and strides as for mla_decode, max_seq_len rows per sequence (>= 64);
  *   o_lat [rows, n_heads, C] bf16 — softmax-weighted sum of cached latents;
  *   lse [rows, n_heads] fp32 or NULL;
- *   status — device int32 or NULL; device-side problems (a start position outside
- *     [0, max_seq_len), a bounded wait that gave up) are recorded there (caller zeroes it).
+ *   status — device int32, required (NULL returns MLA_ERR_INVALID_ARG); the caller zeroes it
+ *     before the call and reads it after synchronising; device-side problems are recorded there:
+ *     6 (MLA_ERR_DEVICE_ARG) for a start position outside [0, max_seq_len), 5
+ *     (MLA_ERR_DEVICE_TIMEOUT) for a bounded wait that gave up.
+ * Argument checks are those of mla_decode (16-byte aligned rows and strides, strides below 2^40
+ * bytes) plus 64 <= max_seq_len <= 2^24.
  * The library uses no memory but its inputs, its outputs and one fixed scratch array of about
  * 4.3 MB that every device loading the library holds until exit.  Limits: rows <= 4096 (more
  * returns MLA_ERR_INVALID_ARG); the split over keys uses at most 16 SM pairs.  The first call on

@@ -14,6 +14,12 @@ from mla_synth import bf16_bits_to_f64, make_inputs, workload
 REL_TOL = 1e-2
 ABS_TOL = 1e-3
 PROB_TOL = 1e-3
+# lse is compared with the oracle run on the same bf16-rounded queries ("bf16" query mode): what
+# is left is fp32 arithmetic on the GPU — scores accumulated in fp32 from bf16 operands (relative
+# error <= 576 * 2^-24 of sum|q_c k_c| * scale, about 4e-4 for these inputs), the hardware exp2 /
+# log2 (relative error ~2^-22) and the fp32 split merge — so 2e-3 absolute is a bound with margin.
+LSE_ATOL = 2e-3
+LSE_RTOL = 0.0
 
 
 def assert_close_bf16(got: np.ndarray, ref: np.ndarray, what: str, rel=REL_TOL, abs_=ABS_TOL):
@@ -66,9 +72,12 @@ def oracle_decode(inp: dict, w, rows=None, **kw):
 
 def oracle_prefill(inp: dict, w, tokens=None, **kw):
     d = w.dims
+    # the chunk's cache prefix is small: widen it once instead of per token
+    n = int(inp["start_pos"][0]) + w.tokens
+    cache = bf16_bits_to_f64(inp["cache"][:, :n])
     return oracle.prefill(
         bf16_bits_to_f64(inp["q_latent"]), inp["gamma"].astype(np.float64),
-        bf16_bits_to_f64(inp["wq_b"]), bf16_bits_to_f64(inp["wkv_b"]), _CacheView(inp["cache"]),
+        bf16_bits_to_f64(inp["wq_b"]), bf16_bits_to_f64(inp["wkv_b"]), cache,
         int(inp["start_pos"][0]), d.n_heads,
         residual=None if inp["residual"] is None else bf16_bits_to_f64(inp["residual"]),
         theta=w.rope_theta, eps=w.rms_eps, tokens=tokens, **kw)
@@ -85,4 +94,5 @@ class _CacheView:
 
 
 __all__ = ["assert_close_bf16", "to_device", "bf16_to_np", "f64", "oracle_decode",
-           "oracle_prefill", "make_inputs", "workload", "REL_TOL", "ABS_TOL", "PROB_TOL"]
+           "oracle_prefill", "make_inputs", "workload", "REL_TOL", "ABS_TOL", "PROB_TOL",
+           "LSE_ATOL", "LSE_RTOL"]

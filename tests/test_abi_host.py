@@ -113,3 +113,29 @@ def test_calls_without_context_rejected(lib):
         mla.mla_prefill_chunk(None, 16, None, 0, 1, 16, 576 * 64, 576, 16, 576 * 64, 576, 1, 16)
     assert mla.mla_sync_status(None) == 1
     assert mla.mla_last_launch_count(None) == 0
+
+
+def test_noalloc_rejects_bad_arguments_before_launching(lib):
+    """The allocation-free entry point checks its arguments on the host like mla_decode: a missing
+    status word, rows beyond its scratch array, unsupported heads, bad strides or sequence lengths
+    return an error before any CUDA call."""
+    ok = dict(q_abs=16, start_pos=16, rows=4, n_heads=128, softmax_scale=0.07, kv_cache=16,
+              kv_stride_b=576 * 64, kv_stride_t=576, pe_cache=16 + 1024, pe_stride_b=576 * 64,
+              pe_stride_t=576, max_seq_len=64, o_lat=16, lse=None, status=16)
+    cases = [
+        (dict(status=None), "MLA_ERR_INVALID_ARG"),
+        (dict(rows=4097), "MLA_ERR_INVALID_ARG"),
+        (dict(rows=0), "MLA_ERR_INVALID_ARG"),
+        (dict(n_heads=24), "MLA_ERR_UNSUPPORTED"),
+        (dict(max_seq_len=32), "MLA_ERR_INVALID_ARG"),
+        (dict(max_seq_len=(1 << 24) + 1), "MLA_ERR_INVALID_ARG"),
+        (dict(kv_stride_t=500), "MLA_ERR_INVALID_ARG"),
+        (dict(kv_stride_b=(1 << 40)), "MLA_ERR_INVALID_ARG"),
+        (dict(pe_cache=18), "MLA_ERR_INVALID_ARG"),
+        (dict(softmax_scale=float("nan")), "MLA_ERR_INVALID_ARG"),
+    ]
+    for change, want in cases:
+        args = {**ok, **change}
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_latent_attention_noalloc(**args)
+        assert mla.STATUS[e.value.status] == want, change

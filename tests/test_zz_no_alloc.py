@@ -1,13 +1,13 @@
-"""The allocation-free attention entry point gives the same result as the context path.
+"""The allocation-free attention entry point matches the oracle on the queries it is given.
 
-Callers that cannot allocate device memory (a fixed pool, a host-imposed budget) use
-mla_latent_attention_noalloc.  This file is named so pytest collects it last; it runs the same
+Callers that cannot allocate device memory where they run (code confined to a fixed pool, a
+plug-in given a device budget by its host) use mla_latent_attention_noalloc.  This file is named so pytest collects it last; it runs the same
 whether started alone in a fresh process or after the other tests.
 """
 import numpy as np
 import pytest
 
-from mla_cases import assert_close_bf16, f64, make_inputs, to_device, workload
+from mla_cases import LSE_ATOL, LSE_RTOL, assert_close_bf16, f64, make_inputs, to_device, workload
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -22,7 +22,10 @@ def _cuda():
 
 
 @pytest.mark.parametrize("H,B,L", [(128, 32, 4096), (64, 5, 300)])
-def test_noalloc_attention_matches_context_path(H, B, L):
+def test_noalloc_attention_matches_oracle(H, B, L):
+    """Absorbed queries come from the context path (they are an input of this entry point); its
+    o_lat and lse are compared with the fp64 oracle's scores, softmax and weighted sum on the same
+    queries, element by element, on two calls in a row that share the scratch array."""
     from head_latent_attention_11_b200 import mla_debug_copy, mla_latent_attention_noalloc
     from head_latent_attention_11_b200.runtime import MLARuntime
     from mla_synth import MLADims
@@ -31,17 +34,26 @@ def test_noalloc_attention_matches_context_path(H, B, L):
     dev = to_device(inp)
     max_t = inp["max_t"]
     stream = torch.cuda.current_stream().cuda_stream
-    # reference: the existing decode entry point, with its absorbed queries and o_lat
     rt = MLARuntime(dev["gamma"], dev["wq_b"], dev["wkv_b"], n_heads=H, max_rows=B,
                     max_seq_len=max_t)
-    lse_ref = torch.empty(B, H, dtype=torch.float32, device="cuda")
-    rt.decode(dev["q_latent"].reshape(B, -1), dev["start_pos"], dev["cache"], lse=lse_ref)
+    rt.decode(dev["q_latent"].reshape(B, -1), dev["start_pos"], dev["cache"])
     q_abs = torch.empty(B, 128, 576, dtype=torch.bfloat16, device="cuda")
-    o_ref = torch.empty(B, H, 512, dtype=torch.bfloat16, device="cuda")
     mla_debug_copy(rt.ctx, 2, q_abs, q_abs.numel() * 2, stream)
-    mla_debug_copy(rt.ctx, 3, o_ref, o_ref.numel() * 2, stream)
     torch.cuda.synchronize()
     assert rt.sync_status() == 0
+    # the oracle's scores, softmax and weighted sum (a5-a7) on exactly these absorbed queries
+    import oracle
+    from mla_synth import bf16_bits_to_f64
+    qa = f64(q_abs)
+    ref_olat = np.empty((B, H, 512))
+    ref_lse = np.empty((B, H))
+    for b in range(B):
+        n = int(inp["start_pos"][b]) + 1
+        rows = bf16_bits_to_f64(inp["cache"][b, :n])
+        s = oracle.latent_scores(qa[b, :H, :512], qa[b, :H, 512:], rows[:, :512], rows[:, 512:],
+                                 192 ** -0.5)
+        p, ref_lse[b] = oracle.softmax_fp(s)
+        ref_olat[b] = oracle.latent_weighted_sum(p, rows[:, :512])
     kv, ksb, kst, pe, psb, pst = rt.cache_views(dev["cache"])
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     for call in range(2):   # two calls in a row share the scratch array
@@ -51,14 +63,15 @@ def test_noalloc_attention_matches_context_path(H, B, L):
                                      psb, pst, max_t, o_lat, lse, status, stream)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
-        assert_close_bf16(f64(o_lat), f64(o_ref), f"o_lat call {call}")
-        np.testing.assert_allclose(lse.cpu().numpy(), lse_ref.cpu().numpy(), atol=2e-3, rtol=1e-4)
+        assert_close_bf16(f64(o_lat), ref_olat, f"o_lat call {call}")
+        np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=LSE_ATOL, rtol=LSE_RTOL)
     rt.close()
 
 
 def test_noalloc_rejects_rows_beyond_scratch():
     from head_latent_attention_11_b200 import MLAError, STATUS, mla_latent_attention_noalloc
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
     with pytest.raises(MLAError) as e:
         mla_latent_attention_noalloc(16, 16, 4097, 128, 0.07, 16, 576 * 64, 576, 16, 576 * 64, 576,
-                                     64, 16)
+                                     64, 16, None, status)
     assert STATUS[e.value.status] == "MLA_ERR_INVALID_ARG"
