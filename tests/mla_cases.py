@@ -83,6 +83,76 @@ def oracle_prefill(inp: dict, w, tokens=None, **kw):
         theta=w.rope_theta, eps=w.rms_eps, tokens=tokens, **kw)
 
 
+# ------------------------------------------------------------------------------------------
+# The oracle over many rows / tokens in worker processes (spawned, so safe after CUDA has been
+# initialised in the test process; each worker uses one BLAS thread)
+# ------------------------------------------------------------------------------------------
+_P_STATE = {}
+
+
+def _pool_init(inp, w):
+    _P_STATE["inp"], _P_STATE["w"] = inp, w
+    try:
+        from threadpoolctl import threadpool_limits
+        _P_STATE["limits"] = threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        pass
+
+
+def _pool_call(task):
+    kind, items, kw = task
+    fn = oracle_decode if kind == "decode" else oracle_prefill
+    key = "rows" if kind == "decode" else "tokens"
+    return fn(_P_STATE["inp"], _P_STATE["w"], **{key: items}, **kw)
+
+
+def _merge(parts, axis):
+    out = {}
+    for k in parts[0]:
+        v = parts[0][k]
+        if isinstance(v, np.ndarray):
+            out[k] = np.concatenate([p[k] for p in parts], axis=axis)
+        elif isinstance(v, list):
+            out[k] = [x for p in parts for x in p[k]]
+        elif v is None:
+            out[k] = None
+        else:
+            raise TypeError(k)
+    return out
+
+
+def oracle_parallel(kind: str, inp: dict, w, items=None, workers=None, **kw):
+    """``oracle_decode`` (kind "decode", items = rows) or ``oracle_prefill`` (kind "prefill",
+    items = tokens) split over worker processes; the result is the same dict the single call
+    returns for all items."""
+    import multiprocessing as mp
+    import os
+    from concurrent.futures import ProcessPoolExecutor
+    n = w.batch if kind == "decode" else w.tokens
+    items = list(range(n)) if items is None else list(items)
+    workers = workers or max(1, min(16, os.cpu_count() or 1, len(items)))
+    chunk = max(1, (len(items) + 4 * workers - 1) // (4 * workers))
+    tasks = [(kind, items[i:i + chunk], kw) for i in range(0, len(items), chunk)]
+    if workers == 1 or len(tasks) == 1:
+        parts = [_pool_call_local(inp, w, t) for t in tasks]
+    else:
+        with ProcessPoolExecutor(workers, mp_context=mp.get_context("spawn"),
+                                 initializer=_pool_init, initargs=(inp, w)) as ex:
+            parts = list(ex.map(_pool_call, tasks))
+    if kind == "decode":
+        return _merge(parts, 0)
+    merged = {"out": np.concatenate([p["out"] for p in parts], axis=1),
+              "lse": np.concatenate([p["lse"] for p in parts], axis=1)}
+    return merged
+
+
+def _pool_call_local(inp, w, task):
+    kind, items, kw = task
+    if kind == "decode":
+        return oracle_decode(inp, w, rows=items, **kw)
+    return oracle_prefill(inp, w, tokens=items, **kw)
+
+
 class _CacheView:
     """Widens rows of the bf16 cache to float64 lazily (indexing [b, :n, cols])."""
 
@@ -95,4 +165,4 @@ class _CacheView:
 
 __all__ = ["assert_close_bf16", "to_device", "bf16_to_np", "f64", "oracle_decode",
            "oracle_prefill", "make_inputs", "workload", "REL_TOL", "ABS_TOL", "PROB_TOL",
-           "LSE_ATOL", "LSE_RTOL"]
+           "LSE_ATOL", "LSE_RTOL", "oracle_parallel"]

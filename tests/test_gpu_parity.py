@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 
 from mla_cases import (LSE_ATOL, LSE_RTOL, PROB_TOL, assert_close_bf16, bf16_to_np, f64,
-                       make_inputs, oracle_decode, oracle_prefill, to_device, workload)
+                       make_inputs, oracle_decode, oracle_parallel, to_device, workload)
 from mla_synth import bf16_bits_to_f64
 
 pytestmark = pytest.mark.gpu
@@ -84,9 +84,10 @@ def _decode_case(w, seed=0, tail="zero", rows=None, check_intermediates=True, ch
                     lse=lse, logits=logits)
     torch.cuda.synchronize()
     assert rt.sync_status() == 0
-    ref = oracle_decode(inp, w, rows=rows,
-                        want_intermediates=check_intermediates or res is not None)
-    refq = oracle_decode(inp, w, rows=rows, want_logits=check_probs, query_precision="bf16")
+    ref = oracle_parallel("decode", inp, w, rows,
+                          want_intermediates=check_intermediates or res is not None)
+    refq = oracle_parallel("decode", inp, w, rows, want_logits=check_probs,
+                           query_precision="bf16")
     sel = np.arange(B) if rows is None else np.asarray(rows)
     got = f64(out)[sel]
     assert_close_bf16(got, ref["out"], f"{w.name} out")
@@ -197,13 +198,16 @@ def _prefill_case(w, seed=0, tokens=None, tail="zero"):
     out = rt.prefill(dev["q_latent"], w.prefill_start, dev["cache"], residual=res, lse=lse)
     torch.cuda.synchronize()
     assert rt.sync_status() == 0
-    ref = oracle_prefill(inp, w, tokens=tokens)
-    refq = oracle_prefill(inp, w, tokens=tokens, query_precision="bf16")
     sel = np.arange(T) if tokens is None else np.asarray(tokens)
-    got = f64(out)[:, sel]
-    assert_close_bf16(got, ref["out"], f"{w.name} out")
-    assert_close_bf16(got, refq["out"], f"{w.name} out (bf16-query oracle)", rel=5e-3)
-    np.testing.assert_allclose(lse.cpu().numpy()[:, sel], refq["lse"], atol=LSE_ATOL,
+    ref = oracle_parallel("prefill", inp, w, sel)
+    # the bf16-query oracle (tighter bound, lse) on every token of small chunks, and on every
+    # 8th token plus the last of large ones
+    selq = sel if len(sel) <= 256 else np.unique(np.concatenate([sel[::8], sel[-1:]]))
+    refq = oracle_parallel("prefill", inp, w, selq, query_precision="bf16")
+    got = f64(out)
+    assert_close_bf16(got[:, sel], ref["out"], f"{w.name} out")
+    assert_close_bf16(got[:, selq], refq["out"], f"{w.name} out (bf16-query oracle)", rel=5e-3)
+    np.testing.assert_allclose(lse.cpu().numpy()[:, selq], refq["lse"], atol=LSE_ATOL,
                                rtol=LSE_RTOL)
     rt.close()
 
