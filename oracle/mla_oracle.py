@@ -48,7 +48,7 @@ import numpy as np
 __all__ = [
     "round_bf16", "rmsnorm", "rope_frequencies", "apply_rope_interleaved", "query_heads", "absorb_w_uk",
     "latent_scores", "softmax_fp", "latent_weighted_sum", "expand_w_uv", "decode", "prefill",
-    "nonabsorbed_attention", "split_wkv_b", "split_wq_b",
+    "nonabsorbed_attention", "split_wkv_b", "split_wq_b", "produce_latents", "write_cache_rows",
 ]
 
 
@@ -307,3 +307,40 @@ def nonabsorbed_attention(q_nope, q_pe, kv, pe, wkv_b, n_heads, *, q_positions, 
         out[:, h] = p @ value
         lse[:, h] = l
     return out, lse
+
+
+# ------------------------------------------------------------------------------------------
+# Cache producer  ([QH] mla-init: wq_a, wkv_a, kv_norm; [QH] mla-queries: qr = q_norm(wq_a(x));
+# [VS] mla-init: the joint key-value down-projection kv_a_proj_with_mqa that also emits the shared
+# rotary key, and its latent RMSNorm kv_a_layernorm)
+# ------------------------------------------------------------------------------------------
+def produce_latents(x, wq_a, wkv_a, kv_norm_gain, pos, *, kv_lora=512, rope=64, theta=10000.0,
+                    eps=1e-6, precision="exact"):
+    """The step upstream of the attention for new tokens ``x`` [M, dim] at positions ``pos`` [M].
+
+    q_latent = x wq_a^T                      (the query latent, input of q_norm)
+    c        = x wkv_a^T  [M, kv_lora + rope] (one Linear: the latent, then the shared rotary key)
+    kv       = RMSNorm(c[:, :kv_lora]) with gain kv_norm_gain (eps 1e-6)
+    k_pe     = RoPE(c[:, kv_lora:], pos)      (interleaved pairs, like q_pe)
+    Returns (q_latent, kv, k_pe).  ``precision="bf16"`` rounds where the pages' tensors are bf16:
+    both Linear outputs, the normalised latent (``.to(dtype)``) and the rotated key."""
+    x = np.asarray(x, np.float64)
+    r = round_bf16 if precision == "bf16" else (lambda a: a)
+    if precision not in ("exact", "bf16"):
+        raise ValueError(precision)
+    q_latent = r(x @ np.asarray(wq_a, np.float64).T)
+    c = r(x @ np.asarray(wkv_a, np.float64).T)
+    kv, _ = rmsnorm(c[:, :kv_lora], kv_norm_gain, eps)
+    k_pe = apply_rope_interleaved(c[:, kv_lora:kv_lora + rope], np.asarray(pos), theta)
+    return q_latent, r(kv), r(k_pe)
+
+
+def write_cache_rows(cache, kv, k_pe, batch_index, pos, kv_lora=512):
+    """Store the new rows: cache[b, pos] = [kv ‖ k_pe] for each new token (the pages write
+    ``kv_cache[:bsz, start_pos:end_pos]`` / ``pe_cache`` before attending over ``:end_pos``).
+    Returns a float64 copy of ``cache`` [B, max_t, kv_lora + rope] with the rows replaced."""
+    out = np.array(cache, dtype=np.float64, copy=True)
+    for i, (b, t) in enumerate(zip(np.asarray(batch_index), np.asarray(pos))):
+        out[b, t, :kv_lora] = kv[i]
+        out[b, t, kv_lora:] = k_pe[i]
+    return out
