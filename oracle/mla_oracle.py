@@ -49,6 +49,7 @@ __all__ = [
     "round_bf16", "rmsnorm", "rope_frequencies", "apply_rope_interleaved", "query_heads", "absorb_w_uk",
     "latent_scores", "softmax_fp", "latent_weighted_sum", "expand_w_uv", "decode", "prefill",
     "nonabsorbed_attention", "split_wkv_b", "split_wq_b", "produce_latents", "write_cache_rows",
+    "index_mask",
 ]
 
 
@@ -166,8 +167,20 @@ def expand_w_uv(o_lat: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
     return np.einsum("...hc,hdc->...hd", o_lat, w_uv)
 
 
-def _attend_row(q_lat_h, q_pe_h, kv, pe, scale, w_uv, want_logits=False):
+def index_mask(topk, end_pos: int) -> np.ndarray:
+    """[AU] mla-decode: ``full((end_pos,), -inf).scatter_(-1, topk_indices, 0)`` — 0 at every
+    selected key, -inf elsewhere.  Entries < 0 are unused slots of a padded index list (this
+    build's convention for rows with fewer than K selected keys)."""
+    m = np.full(end_pos, -np.inf)
+    idx = np.asarray(topk, dtype=np.int64)
+    m[idx[idx >= 0]] = 0.0
+    return m
+
+
+def _attend_row(q_lat_h, q_pe_h, kv, pe, scale, w_uv, want_logits=False, mask=None):
     s = latent_scores(q_lat_h, q_pe_h, kv, pe, scale)
+    if mask is not None:
+        s = s + mask[None, :]
     p, lse = softmax_fp(s)
     o_lat = latent_weighted_sum(p, kv)
     out = expand_w_uv(o_lat, w_uv)
@@ -199,8 +212,11 @@ def _dims(n_heads, nope=128, rope=64, v=128):
 
 def decode(q_latent, gamma, wq_b, wkv_b, cache, start_pos, n_heads, *, residual=None,
            kv_lora=512, nope=128, rope=64, v=128, theta=10000.0, eps=1e-6, scale=None,
-           rows=None, want_logits=False, want_intermediates=False, query_precision="exact"):
-    """Absorbed decode ([AU] mla-decode with the index mask keeping every key).
+           rows=None, want_logits=False, want_intermediates=False, query_precision="exact",
+           topk=None):
+    """Absorbed decode ([AU] mla-decode).  With ``topk`` [B, K] (selected key indices of each
+    sequence) the index mask of the excerpt is added to the scores; without it every key is kept
+    (the mask of a top-k that covers all end_pos keys is all zeros).
 
     ``q_latent`` [B, q_lora]; ``cache`` [B, max_t, kv_lora+rope] (packed latents ‖ pe key);
     ``start_pos`` [B]: sequence b's query is at position start_pos[b] and sees keys 0..start_pos[b].
@@ -221,7 +237,8 @@ def decode(q_latent, gamma, wq_b, wkv_b, cache, start_pos, n_heads, *, residual=
         n = int(pos[i]) + 1
         kv = np.asarray(cache[b, :n, :kv_lora], np.float64)
         pe = np.asarray(cache[b, :n, kv_lora:kv_lora + rope], np.float64)
-        o, lse, s, o_lat = _attend_row(q_lat[i], q_pe[i], kv, pe, scale, w_uv, want_logits)
+        mask = None if topk is None else index_mask(np.asarray(topk)[b], n)
+        o, lse, s, o_lat = _attend_row(q_lat[i], q_pe[i], kv, pe, scale, w_uv, want_logits, mask)
         outs.append(o)
         lses.append(lse)
         logits.append(s)
