@@ -49,7 +49,7 @@ __all__ = [
     "round_bf16", "rmsnorm", "rope_frequencies", "apply_rope_interleaved", "query_heads", "absorb_w_uk",
     "latent_scores", "softmax_fp", "latent_weighted_sum", "expand_w_uv", "decode", "prefill",
     "nonabsorbed_attention", "split_wkv_b", "split_wq_b", "produce_latents", "write_cache_rows",
-    "index_mask",
+    "index_mask", "output_projection", "nonabsorbed_prefill",
 ]
 
 
@@ -361,3 +361,46 @@ def write_cache_rows(cache, kv, k_pe, batch_index, pos, kv_lora=512):
         out[b, t, :kv_lora] = kv[i]
         out[b, t, kv_lora:] = k_pe[i]
     return out
+
+
+# ------------------------------------------------------------------------------------------
+# Output projection and the non-absorbed prefill  ([AU] mla-output: x = wo(x.flatten(2));
+# [VS] mla-prefill: per-head keys and values rebuilt from the latent, additive causal mask)
+# ------------------------------------------------------------------------------------------
+def output_projection(o, wo):
+    """wo applied to the flattened head outputs: ``o`` [..., H, v] → [..., dim] with
+    y[..., i] = sum_{h, d} wo[i, h*v + d] * o[..., h, d] (wo in nn.Linear layout [dim, H*v])."""
+    o = np.asarray(o, np.float64)
+    flat = o.reshape(o.shape[:-2] + (o.shape[-2] * o.shape[-1],))
+    return flat @ np.asarray(wo, np.float64).T
+
+
+def nonabsorbed_prefill(q_latent, gamma, wq_b, wkv_b, cache, start_pos, n_heads, wo=None, *,
+                        residual=None, kv_lora=512, nope=128, rope=64, v=128, theta=10000.0,
+                        eps=1e-6, scale=None, tokens=None):
+    """A prefill chunk in the pages' other form: the query as in the absorbed path (q_norm, wq_b,
+    RoPE), then for every head the keys [W_UK kv ‖ pe] and values W_UV kv rebuilt from the latent
+    cache, causal softmax attention with the additive mask, and (with ``wo``) the output
+    projection.  ``q_latent`` [B, T, q_lora]; returns ``out`` [B, T', H, v], ``lse`` [B, T', H]
+    and ``y`` [B, T', dim] when ``wo`` is given."""
+    q_latent = np.asarray(q_latent, np.float64)
+    B, T, _ = q_latent.shape
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    dims = _dims(n_heads, nope, rope, v)
+    out = np.empty((B, len(tokens), n_heads, v))
+    lse = np.empty((B, len(tokens), n_heads))
+    for b in range(B):
+        rs = None if residual is None else np.asarray(residual, np.float64)[b, tokens]
+        pos = int(start_pos) + tokens.astype(np.int64)
+        _, _, q_nope, q_pe, _, _ = _front(q_latent[b, tokens], rs, gamma, wq_b, wkv_b, dims, pos,
+                                          theta, eps)
+        n = int(pos.max()) + 1
+        kv = np.asarray(cache[b, :n, :kv_lora], np.float64)
+        pe = np.asarray(cache[b, :n, kv_lora:kv_lora + rope], np.float64)
+        o, l = nonabsorbed_attention(q_nope, q_pe, kv, pe, wkv_b, n_heads, q_positions=pos,
+                                     nope=nope, v=v, scale=scale)
+        out[b], lse[b] = o, l
+    r = {"out": out, "lse": lse}
+    if wo is not None:
+        r["y"] = output_projection(out, wo)
+    return r
