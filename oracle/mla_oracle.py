@@ -49,7 +49,8 @@ __all__ = [
     "round_bf16", "rmsnorm", "rope_frequencies", "apply_rope_interleaved", "query_heads", "absorb_w_uk",
     "latent_scores", "softmax_fp", "latent_weighted_sum", "expand_w_uv", "decode", "prefill",
     "nonabsorbed_attention", "split_wkv_b", "split_wq_b", "produce_latents", "write_cache_rows",
-    "index_mask", "output_projection", "nonabsorbed_prefill",
+    "index_mask", "output_projection", "nonabsorbed_prefill", "fp8_e4m3_value",
+    "dequant_block_fp8",
 ]
 
 
@@ -404,3 +405,31 @@ def nonabsorbed_prefill(q_latent, gamma, wq_b, wkv_b, cache, start_pos, n_heads,
     if wo is not None:
         r["y"] = output_projection(out, wo)
     return r
+
+
+# ------------------------------------------------------------------------------------------
+# FP8 block-scaled weights  ([AU] mla-decode: ``weight_dequant(self.wkv_b.weight,
+# self.wkv_b.scale)``; [QH] parameter table note: the checkpoint stores FP8 weights with block
+# scales)
+# ------------------------------------------------------------------------------------------
+def fp8_e4m3_value(bits) -> np.ndarray:
+    """Value of FP8 E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; exponent
+    field 0 is subnormal: m/8 * 2^-6; no infinities; S.1111.111 is NaN) as float64."""
+    b = np.asarray(bits, dtype=np.int64) & 0xFF
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 0x7).astype(np.float64)
+    normal = (1.0 + m / 8.0) * np.power(2.0, e - 7.0)
+    sub = (m / 8.0) * 2.0 ** -6
+    v = sign * np.where(e == 0, sub, normal)
+    return np.where((b & 0x7F) == 0x7F, np.nan, v)
+
+
+def dequant_block_fp8(bits, scale, block: int = 128) -> np.ndarray:
+    """weight_dequant: w[i, j] = value(bits[i, j]) * scale[i // block, j // block], returned in
+    the default dtype (bf16) as the pages' decode uses it — rounded to bf16 here, as float64."""
+    v = fp8_e4m3_value(bits)
+    s = np.asarray(scale, np.float64)
+    rows = np.arange(v.shape[0]) // block
+    cols = np.arange(v.shape[1]) // block
+    return round_bf16(v * s[rows][:, cols])
