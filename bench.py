@@ -43,22 +43,33 @@ METRIC = "MLA decode queries/s + HBM GB/s (% peak); prefill-chunk TFLOP/s (% pea
 FLUSH_BYTES = 256 << 20
 HEADLINE = "ragged_decode"
 WORKLOAD_ORDER = ("ragged_decode", "tiny_decode", "v32_decode", "prefill_chunk", "kimi_decode")
+# variants of the path measured beside the configurations: name -> (workload, variant)
+VARIANTS = {"v32_decode_fp8": ("v32_decode", "fp8"),
+            "ragged_decode_top2048": ("ragged_decode", "top2048")}
 
 
 # ------------------------------------------------------------------------------------------
 # Algorithmic work of one step (bytes the method must move, flops it must do)
 # ------------------------------------------------------------------------------------------
-def algorithmic_work(w, start_pos: np.ndarray) -> dict:
+def algorithmic_work(w, start_pos: np.ndarray, fp8: bool = False, topk_len=None) -> dict:
+    """Bytes and flops of one step.  ``fp8``: weights are one-byte codes plus one fp32 scale per
+    128 x 128 block.  ``topk_len``: index-mask decode, row b attends topk_len[b] keys."""
     d = w.dims
     H, R, C, Dn, Dr, Dv = d.n_heads, d.q_lora_rank, d.kv_lora_rank, d.qk_nope_head_dim, d.qk_rope_head_dim, d.v_head_dim
     rows = w.batch * w.tokens
     keys = keys_per_row(w, start_pos)                      # [B, T] visible keys per query row
+    if topk_len is not None:
+        keys = np.asarray(topk_len, np.int64)[:, None]
     if w.mode == "decode":
         cache_rows = int(keys.sum())                       # each decode row reads its own keys
     else:
         cache_rows = int(keys[:, -1].sum())                # a chunk reads its cache prefix once
     act = rows * R * 2 * (3 if w.residual else 1) + rows * R * 2   # x (+res r/w) + y
-    weights = H * (Dn + Dr) * R * 2 + H * (Dn + Dv) * C * 2 + R * 4
+    if fp8:
+        weights = (H * (Dn + Dr) * R + H * (Dn + Dv) * C
+                   + (H * (Dn + Dr) * R + H * (Dn + Dv) * C) // (128 * 128) * 4 + R * 4)
+    else:
+        weights = H * (Dn + Dr) * R * 2 + H * (Dn + Dv) * C * 2 + R * 4
     cache = cache_rows * (C + Dr) * 2
     out = rows * H * Dv * 2
     flops = (2 * rows * R * H * (Dn + Dr) + 2 * rows * H * Dn * C
@@ -229,9 +240,12 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------
 # Our arm
 # ------------------------------------------------------------------------------------------
-def run_workload(name: str, args, rank: int, world: int, local_rank: int) -> dict | None:
+def run_workload(name: str, args, rank: int, world: int, local_rank: int,
+                 variant: str | None = None, entry: str | None = None) -> dict | None:
     """Times one configuration on this rank's GPU; returns its JSON entry on rank 0 (None on the
-    other ranks).  Every rank takes the same collective steps (two barriers, one all-reduce)."""
+    other ranks).  Every rank takes the same collective steps (two barriers, one all-reduce).
+    ``variant``: "fp8" (FP8 block-scaled weights) or "top2048" (index-mask decode, 2048 seeded
+    selected keys per sequence)."""
     import torch
     import torch.distributed as dist
 
@@ -239,10 +253,13 @@ def run_workload(name: str, args, rank: int, world: int, local_rank: int) -> dic
     from head_latent_attention_11_b200 import (mla_enable_stage_timing, mla_last_launch_count,
                                                mla_stage_times)
     from head_latent_attention_11_b200.runtime import MLARuntime
+    from mla_synth import make_fp8_weights, make_topk
 
     w = workload(name)
     inp = make_inputs(w, seed=args.seed + rank)
-    work = algorithmic_work(w, inp["start_pos"])
+    topk = make_topk(inp["start_pos"], 2048, seed=args.seed + rank) if variant == "top2048" else None
+    work = algorithmic_work(w, inp["start_pos"], fp8=variant == "fp8",
+                            topk_len=None if topk is None else topk[1])
     B, T, H = w.batch, w.tokens, w.dims.n_heads
 
     def bf16(a):
@@ -255,11 +272,22 @@ def run_workload(name: str, args, rank: int, world: int, local_rank: int) -> dic
     if residual is not None and w.mode == "decode":
         residual = residual.reshape(B, -1)
     gamma = torch.from_numpy(inp["gamma"]).to(dev)
-    wq_b, wkv_b, cache = bf16(inp["wq_b"]), bf16(inp["wkv_b"]), bf16(inp["cache"])
+    cache = bf16(inp["cache"])
     start_pos = torch.from_numpy(inp["start_pos"].astype(np.int32)).to(dev)
+    scales = {}
+    if variant == "fp8":
+        f8 = make_fp8_weights(w, seed=args.seed + rank)
+        wq_b, wkv_b = torch.from_numpy(f8["wq_b"]).to(dev), torch.from_numpy(f8["wkv_b"]).to(dev)
+        scales = dict(wq_b_scale=torch.from_numpy(f8["wq_b_scale"]).to(dev),
+                      wkv_b_scale=torch.from_numpy(f8["wkv_b_scale"]).to(dev))
+    else:
+        wq_b, wkv_b = bf16(inp["wq_b"]), bf16(inp["wkv_b"])
+    t_idx = t_len = None
+    if topk is not None:
+        t_idx, t_len = torch.from_numpy(topk[0]).to(dev), torch.from_numpy(topk[1]).to(dev)
     del inp
     rt = MLARuntime(gamma, wq_b, wkv_b, n_heads=H, max_rows=B * T, max_seq_len=cache.shape[1],
-                    rope_theta=w.rope_theta, rms_eps=w.rms_eps)
+                    rope_theta=w.rope_theta, rms_eps=w.rms_eps, **scales)
     out_shape = (B, H, 128) if w.mode == "decode" else (B, T, H, 128)
     out = torch.empty(out_shape, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -274,12 +302,16 @@ def run_workload(name: str, args, rank: int, world: int, local_rank: int) -> dic
         flush.fill_(float(i))   # evict everything the previous step left in L2 ...
         flush_rd.sum()          # ... and leave L2 holding clean lines of an unrelated buffer
 
-    def step():
-        if w.mode == "decode":
-            rt.decode(q_latent, start_pos, cache, residual=residual, out=out, stream=stream)
+    def step(q_in=None, sp=None):
+        q_in = q_latent if q_in is None else q_in
+        sp = start_pos if sp is None else sp
+        if topk is not None:
+            rt.decode_sparse(q_in, sp, t_idx, t_len, cache, residual=residual, out=out,
+                             stream=stream)
+        elif w.mode == "decode":
+            rt.decode(q_in, sp, cache, residual=residual, out=out, stream=stream)
         else:
-            rt.prefill(q_latent, w.prefill_start, cache, residual=residual, out=out,
-                       stream=stream)
+            rt.prefill(q_in, w.prefill_start, cache, residual=residual, out=out, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -357,10 +389,7 @@ def run_workload(name: str, args, rank: int, world: int, local_rank: int) -> dic
         e0.record(stream)
         d_q.copy_(h_q, non_blocking=True)
         d_sp.copy_(h_sp, non_blocking=True)
-        if w.mode == "decode":
-            rt.decode(d_q, d_sp, cache, residual=residual, out=out, stream=stream)
-        else:
-            rt.prefill(d_q, w.prefill_start, cache, residual=residual, out=out, stream=stream)
+        step(d_q, d_sp)
         h_out.copy_(out, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
@@ -393,7 +422,7 @@ def run_workload(name: str, args, rank: int, world: int, local_rank: int) -> dic
         achieved = work["attn_bytes"] / (attn_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": profiled_traffic(w.name), "kernel": "latent_attention",
+                "traffic": profiled_traffic(entry or w.name), "kernel": "latent_attention",
                 "algorithmic_bytes_per_launch": work["attn_bytes"],
                 "algorithmic_bytes_rule": "cache rows attended x 1152 B (576 bf16)",
                 "kernel_ms": round(attn_ms, 5),
@@ -410,7 +439,9 @@ def run_workload(name: str, args, rank: int, world: int, local_rank: int) -> dic
     step_gbs = work["bytes"] / (ms_per_step / 1e3) / 1e9
     return {
         "value": round(value, 2), "unit": unit, "ms_per_step": round(ms_per_step, 5),
-        "config": {"workload": w.name, "batch": B, "tokens": T, "n_heads": H,
+        "config": {"workload": entry or w.name, "batch": B, "tokens": T, "n_heads": H,
+                   "weights": "fp8 e4m3, 128x128 block scales" if variant == "fp8" else "bf16",
+                   "keys": "2048 selected per sequence (index mask)" if topk is not None else "all",
                    "cache_keys_per_step": work["keys"], "q_lora": 1536, "kv_lora": 512,
                    "rope": 64, "v": 128, "residual": bool(w.residual),
                    "l2": "flushed before every timed step: 256 MiB write, then 256 MiB read of another buffer (untimed)",
@@ -428,6 +459,221 @@ def run_workload(name: str, args, rank: int, world: int, local_rank: int) -> dic
         "gpu_launches": launches * args.steps,
         "kernels_per_step": launches,
     }
+
+
+# ------------------------------------------------------------------------------------------
+# The cache producer (wq_a, wkv_a → kv_norm / key RoPE → cache rows), upstream of the path
+# ------------------------------------------------------------------------------------------
+PRODUCER_RUNS = {"cache_producer_decode": "v32_decode", "cache_producer_chunk": "prefill_chunk"}
+
+
+def producer_work(w, dim: int) -> dict:
+    d = w.dims
+    rows = w.batch * w.tokens
+    weights = (d.q_lora_rank + d.cache_width) * dim * 2 + d.kv_lora_rank * 4
+    x = rows * dim * 2
+    q_out = rows * d.q_lora_rank * 2
+    cache_rows = rows * d.cache_width * 2
+    flops = 2 * rows * dim * (d.q_lora_rank + d.cache_width)
+    wq_a_bytes = d.q_lora_rank * dim * 2 + x + q_out           # the dominant (first) GEMM
+    wq_a_flops = 2 * rows * dim * d.q_lora_rank
+    return dict(bytes=weights + x + q_out + cache_rows, flops=flops, rows=rows,
+                wq_a_bytes=wq_a_bytes, wq_a_flops=wq_a_flops)
+
+
+def run_producer(name: str, args, rank: int, world: int, local_rank: int) -> dict | None:
+    import torch
+    import torch.distributed as dist
+    from mla_synth import MODEL_DIM, make_producer_inputs
+
+    dev = f"cuda:{local_rank}"
+    from head_latent_attention_11_b200 import (mla_enable_stage_timing, mla_last_launch_count,
+                                               mla_stage_times)
+    from head_latent_attention_11_b200.runtime import MLARuntime
+
+    w = workload(PRODUCER_RUNS[name])
+    inp = make_inputs(w, seed=args.seed + rank)
+    pin = make_producer_inputs(w, seed=args.seed + rank, dim=MODEL_DIM)
+    work = producer_work(w, MODEL_DIM)
+    B, T = w.batch, w.tokens
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    gamma = torch.from_numpy(inp["gamma"]).to(dev)
+    wq_b, wkv_b, cache = bf16(inp["wq_b"]), bf16(inp["wkv_b"]), bf16(inp["cache"])
+    start_pos = torch.from_numpy(inp["start_pos"].astype(np.int32)).to(dev)
+    x = bf16(pin["x"])
+    wq_a, wkv_a = bf16(pin["wq_a"]), bf16(pin["wkv_a"])
+    kv_gain = torch.from_numpy(pin["kv_gain"]).to(dev)
+    del inp, pin
+    rt = MLARuntime(gamma, wq_b, wkv_b, n_heads=w.dims.n_heads, max_rows=B * T,
+                    max_seq_len=cache.shape[1], rope_theta=w.rope_theta, rms_eps=w.rms_eps)
+    rt.attach_producer(wq_a, wkv_a, kv_gain)
+    q_lat = torch.empty(B, T, 1536, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    prev_stream = torch.cuda.current_stream(dev)
+    torch.cuda.set_stream(stream)
+
+    def flush_l2(i: int) -> None:
+        flush.fill_(float(i))
+        flush_rd.sum()
+
+    def step(xin=x, sp=start_pos):
+        if w.mode == "decode":
+            rt.produce(xin, cache, start_pos=sp, q_latent=q_lat, stream=stream)
+        else:
+            rt.produce(xin, cache, start_pos_host=w.prefill_start, q_latent=q_lat, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if rt.sync_status(stream) != 0:
+        raise RuntimeError(f"{name}: device status set during warm-up")
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        graph.replay()
+        torch.cuda.synchronize()
+    run_step = graph.replay if graph is not None else step
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    clocks.mark("load")
+    t_load = time.perf_counter()
+    while time.perf_counter() - t_load < 0.5:
+        for i in range(16):
+            flush_l2(i)
+            run_step()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.mark("timed0")
+    for i in range(args.steps):
+        flush_l2(i)
+        starts[i].record(stream)
+        run_step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clocks.mark("timed1")
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    launches = mla_last_launch_count(rt.ctx)
+    if rt.sync_status(stream) != 0:
+        raise RuntimeError(f"{name}: device status set during the timed steps")
+    total_ms = float(sum(s_.elapsed_time(e) for s_, e in zip(starts, ends)))
+    mla_enable_stage_timing(rt.ctx, True)
+    stage_acc: dict[str, list[float]] = {}
+    for i in range(max(3, min(args.steps, 20))):
+        flush_l2(i)
+        step()
+        for kname, ms in mla_stage_times(rt.ctx):
+            stage_acc.setdefault(kname, []).append(ms)
+    mla_enable_stage_timing(rt.ctx, False)
+    stages = {k: float(np.mean(v)) for k, v in stage_acc.items()}
+    # end to end: x and positions from pinned host memory, the query latent back to the host
+    h_x = torch.empty(x.shape, dtype=torch.bfloat16, pin_memory=True)
+    h_x.copy_(x.cpu())
+    h_sp = torch.empty(start_pos.shape, dtype=torch.int32, pin_memory=True)
+    h_sp.copy_(start_pos.cpu())
+    h_q = torch.empty(q_lat.shape, dtype=torch.bfloat16, pin_memory=True)
+    d_x, d_sp = torch.empty_like(x), torch.empty_like(start_pos)
+    e2e_ms = []
+    for i in range(args.steps):
+        flush_l2(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        d_x.copy_(h_x, non_blocking=True)
+        d_sp.copy_(h_sp, non_blocking=True)
+        step(d_x, d_sp)
+        h_q.copy_(q_lat, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    h2d = h_x.numel() * 2 + h_sp.numel() * 4
+    d2h = h_q.numel() * 2
+    total_ms, e2e_total = max_over_ranks([total_ms, float(np.sum(e2e_ms))], device=dev)
+    rt.close()
+    torch.cuda.set_stream(prev_stream)
+    del graph, rt, cache, wq_b, wkv_b, wq_a, wkv_a, flush, flush_rd
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    if rank != 0:
+        return None
+    peaks = measured_peaks()
+    ms_per_step = total_ms / args.steps
+    rows = work["rows"]
+    value = aggregate_throughput(rows, args.steps, world, total_ms)
+    e2e_value = aggregate_throughput(rows, args.steps, world, e2e_total)
+    k_ms = stages.get("wq_a")
+    if w.mode == "decode":
+        achieved = work["wq_a_bytes"] / (k_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "kernel": "wq_a GEMM", "algorithmic_bytes_per_launch": work["wq_a_bytes"],
+                "algorithmic_bytes_rule": "wq_a weights + x + q_latent out",
+                "kernel_ms": round(k_ms, 5),
+                "peak_source": peaks["source"] + " (hbm_gbs, copy burst)"}
+    else:
+        achieved = work["wq_a_flops"] / (k_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "traffic": None, "kernel": "wq_a GEMM",
+                "algorithmic_flops_per_launch": work["wq_a_flops"],
+                "algorithmic_flops_rule": "2 x tokens x 7168 x 1536",
+                "kernel_ms": round(k_ms, 5),
+                "peak_source": peaks["source"] + " (bf16_tflops, burst)"}
+    step_gbs = work["bytes"] / (ms_per_step / 1e3) / 1e9
+    return {
+        "value": round(value, 2), "unit": "tokens/s", "ms_per_step": round(ms_per_step, 5),
+        "config": {"workload": name, "batch": B, "tokens": T, "dim": MODEL_DIM,
+                   "writes": "kv_cache / pe_cache rows at each token's position",
+                   "l2": "flushed before every timed step (untimed)",
+                   "launch": "CUDA graph of one C-ABI call" if not args.no_graph else "eager C-ABI call",
+                   "parallelism": f"replicas x{world}"},
+        "hbm": {"step_bytes": work["bytes"], "step_gbs": round(step_gbs, 1),
+                "frac_of_peak": round(step_gbs / peaks["hbm_gbs"], 4)},
+        "tflops_step": round(work["flops"] / (ms_per_step / 1e3) / 1e12, 2),
+        "roofline": roof,
+        "stages_ms": {k: round(v, 5) for k, v in stages.items()},
+        "clocks": clk,
+        "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_total / args.steps, 5)},
+        "gpu_launches": launches * args.steps,
+        "kernels_per_step": launches,
+    }
+
+
+def producer_oracle_sample(name: str, budget_s: float) -> dict:
+    from mla_synth import MODEL_DIM, bf16_bits_to_f64, make_producer_inputs
+    import oracle
+    w = workload(PRODUCER_RUNS[name])
+    pin = make_producer_inputs(w, seed=0, dim=MODEL_DIM)
+    x = bf16_bits_to_f64(pin["x"]).reshape(w.batch * w.tokens, -1)
+    wq_a, wkv_a = bf16_bits_to_f64(pin["wq_a"]), bf16_bits_to_f64(pin["wkv_a"])
+    gain = pin["kv_gain"].astype(np.float64)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        cores = 1
+    done, t0 = 0, time.perf_counter()
+    while True:
+        r = done % x.shape[0]
+        oracle.produce_latents(x[r:r + 1], wq_a, wkv_a, gain, np.array([r]))
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    return dict(value=round(done / el, 4), unit="tokens/s", cores=cores, kind="oracle",
+                sample=f"{done} single-token producer calls (cycling over {x.shape[0]} tokens) in {el:.1f} s")
 
 
 # ------------------------------------------------------------------------------------------
@@ -535,6 +781,12 @@ def main(argv=None):
 
     names = WORKLOAD_ORDER if args.workload == "all" else (args.workload,)
     entries = {n: run_workload(n, args, rank, world, local_rank) for n in names}
+    if args.workload == "all":
+        for n, (base, variant) in VARIANTS.items():
+            entries[n] = run_workload(base, args, rank, world, local_rank, variant=variant,
+                                      entry=n)
+        for n in PRODUCER_RUNS:
+            entries[n] = run_producer(n, args, rank, world, local_rank)
     if rank == 0:
         head_name = names[0]
         head = entries[head_name]
@@ -553,11 +805,14 @@ def main(argv=None):
                     "U(0.5,1.5) gain)",
         }
         line.update({k: v for k, v in head.items() if k not in ("value", "unit", "ms_per_step")})
-        line["gpu_launches"] = sum(e["gpu_launches"] for e in entries.values())
+        line["gpu_launches"] = sum(e["gpu_launches"] for e in entries.values() if e)
         line["gpu_launches_note"] = ("kernels of this library launched in the timed steps of "
                                      "every workload below (headline included)")
+        if not args.no_cpu_baseline and world == 1 and args.workload == "all":
+            for n in PRODUCER_RUNS:
+                entries[n]["cpu_baseline"] = producer_oracle_sample(n, min(4.0, args.cpu_seconds))
         if len(names) > 1:
-            line["workloads"] = {n: entries[n] for n in names[1:]}
+            line["workloads"] = {n: entries[n] for n in entries if n != head_name}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

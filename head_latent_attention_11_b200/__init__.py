@@ -18,7 +18,9 @@ __all__ = [
     "MLAError", "MLAConfig", "load", "lib_path", "mla_status_string", "mla_workspace_size",
     "mla_init", "mla_destroy", "mla_rmsnorm", "mla_decode", "mla_prefill_chunk", "mla_sync_status",
     "mla_enable_stage_timing", "mla_stage_times", "mla_debug_copy", "mla_last_launch_count",
-    "EXPORTED_SYMBOLS", "STATUS", "mla_latent_attention_noalloc",
+    "EXPORTED_SYMBOLS", "STATUS", "mla_latent_attention_noalloc", "mla_attach_producer",
+    "mla_produce", "mla_decode_sparse", "mla_init_fp8", "mla_mha_scratch_size",
+    "mla_prefill_chunk_mha", "mla_set_wait_limit",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,7 +35,8 @@ EXPORTED_SYMBOLS = (
     "mla_status_string", "mla_workspace_size", "mla_init", "mla_destroy", "mla_rmsnorm",
     "mla_decode", "mla_prefill_chunk", "mla_sync_status", "mla_enable_stage_timing",
     "mla_stage_times", "mla_debug_copy", "mla_last_launch_count",
-    "mla_latent_attention_noalloc",
+    "mla_latent_attention_noalloc", "mla_attach_producer", "mla_produce", "mla_decode_sparse",
+    "mla_init_fp8", "mla_mha_scratch_size", "mla_prefill_chunk_mha", "mla_set_wait_limit",
 )
 
 
@@ -99,6 +102,16 @@ def load() -> ctypes.CDLL:
         "mla_last_launch_count": (I32, [P]),
         "mla_latent_attention_noalloc": (ctypes.c_int, [P, P, I32, I32, F, P, I64, I64, P, I64,
                                                         I64, I32, P, P, P, P]),
+        "mla_attach_producer": (ctypes.c_int, [P, I32, P, P, P]),
+        "mla_mha_scratch_size": (SZ, [P, I32, I32, I32]),
+        "mla_set_wait_limit": (ctypes.c_int, [P, ctypes.c_uint64]),
+        "mla_prefill_chunk_mha": (ctypes.c_int, [P, P, P, I32, I32, P, I64, I64, P, I64, I64, I32,
+                                                 P, SZ, P, P, P, I32, P, P]),
+        "mla_init_fp8": (ctypes.c_int, [ctypes.POINTER(MLAConfig), P, P, P, P, P, P, SZ, P,
+                                        ctypes.POINTER(P)]),
+        "mla_decode_sparse": (ctypes.c_int, [P, P, P, P, P, P, I32, P, I64, I64, P, I64, I64, I32,
+                                             P, P, P]),
+        "mla_produce": (ctypes.c_int, [P, P, P, I32, I32, I32, P, I64, I64, P, I64, I64, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -213,3 +226,52 @@ def mla_latent_attention_noalloc(q_abs, start_pos, rows: int, n_heads: int, soft
         _ptr(q_abs), _ptr(start_pos), rows, n_heads, softmax_scale, _ptr(kv_cache), kv_stride_b,
         kv_stride_t, _ptr(pe_cache), pe_stride_b, pe_stride_t, max_seq_len, _ptr(o_lat),
         _ptr(lse), _ptr(status), _stream(stream)))
+
+
+def mla_attach_producer(ctx, dim: int, wq_a, wkv_a, kv_norm_gain) -> None:
+    _check("mla_attach_producer", load().mla_attach_producer(ctx, dim, _ptr(wq_a), _ptr(wkv_a),
+                                                             _ptr(kv_norm_gain)))
+
+
+def mla_produce(ctx, x, start_pos, start_pos_host: int, T: int, B: int, kv_cache, kv_stride_b: int,
+                kv_stride_t: int, pe_cache, pe_stride_b: int, pe_stride_t: int, q_latent,
+                stream=None) -> None:
+    _check("mla_produce", load().mla_produce(
+        ctx, _ptr(x), _ptr(start_pos), start_pos_host, T, B, _ptr(kv_cache), kv_stride_b,
+        kv_stride_t, _ptr(pe_cache), pe_stride_b, pe_stride_t, _ptr(q_latent), _stream(stream)))
+
+
+def mla_decode_sparse(ctx, q_latent, residual, start_pos, topk_idx, topk_len, k: int, kv_cache,
+                      kv_stride_b: int, kv_stride_t: int, pe_cache, pe_stride_b: int,
+                      pe_stride_t: int, B: int, out, lse=None, stream=None) -> None:
+    _check("mla_decode_sparse", load().mla_decode_sparse(
+        ctx, _ptr(q_latent), _ptr(residual), _ptr(start_pos), _ptr(topk_idx), _ptr(topk_len), k,
+        _ptr(kv_cache), kv_stride_b, kv_stride_t, _ptr(pe_cache), pe_stride_b, pe_stride_t, B,
+        _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def mla_init_fp8(cfg: MLAConfig, q_norm_gain, wq_b_fp8, wq_b_scale, wkv_b_fp8, wkv_b_scale,
+                 workspace, workspace_bytes: int, stream=None) -> ctypes.c_void_p:
+    ctx = ctypes.c_void_p()
+    _check("mla_init_fp8", load().mla_init_fp8(
+        ctypes.byref(cfg), _ptr(q_norm_gain), _ptr(wq_b_fp8), _ptr(wq_b_scale), _ptr(wkv_b_fp8),
+        _ptr(wkv_b_scale), _ptr(workspace), workspace_bytes, _stream(stream), ctypes.byref(ctx)))
+    return ctx
+
+
+def mla_mha_scratch_size(ctx, B: int, T: int, start_pos: int) -> int:
+    return int(load().mla_mha_scratch_size(ctx, B, T, start_pos))
+
+
+def mla_prefill_chunk_mha(ctx, q_latent, residual, start_pos: int, T: int, kv_cache,
+                          kv_stride_b: int, kv_stride_t: int, pe_cache, pe_stride_b: int,
+                          pe_stride_t: int, B: int, kv_scratch, scratch_bytes: int, out, lse=None,
+                          wo=None, dim: int = 0, y=None, stream=None) -> None:
+    _check("mla_prefill_chunk_mha", load().mla_prefill_chunk_mha(
+        ctx, _ptr(q_latent), _ptr(residual), start_pos, T, _ptr(kv_cache), kv_stride_b,
+        kv_stride_t, _ptr(pe_cache), pe_stride_b, pe_stride_t, B, _ptr(kv_scratch), scratch_bytes,
+        _ptr(out), _ptr(lse), _ptr(wo), dim, _ptr(y), _stream(stream)))
+
+
+def mla_set_wait_limit(ctx, ns: int) -> None:
+    _check("mla_set_wait_limit", load().mla_set_wait_limit(ctx, int(ns)))

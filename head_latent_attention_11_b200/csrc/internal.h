@@ -21,7 +21,7 @@ constexpr int kDq = kDn + kDr;        // 192 query features per head
 constexpr int kDk = kC + kDr;         // 576-wide absorbed query / cache row
 constexpr int kHPad = 128;            // heads padded to one 128-row MMA tile
 constexpr int kRopePairs = kDr / 2;   // 32
-constexpr int kAttnKeysPerTile = 32;  // cache rows per attention tile (TMA box height)
+constexpr int kAttnKeysPerTile = 64;  // cache rows per attention tile (TMA box height)
 
 // ---------------------------------------------------------------------------------------
 // a1: RMSNorm (+ residual) with the rotary table and the per-row key prefix as side outputs
@@ -52,6 +52,28 @@ struct RmsParams {
   int2* row_pieces;         // [rows]
   int n_pairs;
   int min_keys_per_pair;
+  int* status;
+  // index-mask decode: per-row count of selected keys (null: dense) and the list capacity K
+  const int32_t* topk_len;
+  int topk_k;
+};
+
+// ---------------------------------------------------------------------------------------
+// Cache producer: kv_norm + key RoPE of the wkv_a output, written to the caller's cache rows
+// ---------------------------------------------------------------------------------------
+struct KvFinishParams {
+  const bf16* c;            // [rows, 576]: wkv_a output (latent ‖ rotary key), bf16
+  const float* gain;        // [512] kv_norm gain
+  bf16* kv_cache;           // row of key t of sequence b at kv_cache + b*kv_sb + t*kv_st
+  long long kv_sb, kv_st;
+  bf16* pe_cache;
+  long long pe_sb, pe_st;
+  int rows, T;              // row = b*T + t
+  const int32_t* start_pos_dev;   // [B] or null (then start_pos for every sequence)
+  int start_pos;
+  int max_seq_len;
+  float eps;
+  double rope_log_theta;
   int* status;
 };
 
@@ -84,7 +106,33 @@ struct GemmParams {
   bf16* o_lat;                  // [rows, n_heads, 512]
   float* lse_out;               // [rows, n_heads] or null
   int n_pairs, min_keys_per_pair;
+  // FP8 E4M3 weights (null: bf16 A): A holds fp8 codes; the value of A[g][m][k] is its code times
+  // a_scale[g * a_sg + ((m + a_row_off) / 128) * a_sm + (k / 128) * a_sk] (128 x 128 blocks)
+  const float* a_scale;
+  long long a_sg, a_sm, a_sk;
+  int b_g0;                // B is shared by every batch g (its batch coordinate is 0)
+  unsigned long long wait_limit_ns;   // bound of every wait in the kernel (0: the 2 s default)
 };
+
+// ---------------------------------------------------------------------------------------
+// Non-absorbed prefill: multi-head attention over keys / values rebuilt from the latent
+// ---------------------------------------------------------------------------------------
+struct FmhaParams {
+  bf16* out;              // [B*T, H, 128]
+  float* lse;             // [B*T, H] or null
+  int T, B, n_heads, start_pos;
+  float scale_log2;
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+struct FmhaMaps {
+  CUtensorMap qn;         // q_nope {128, H, rows},           box {64, 1, 128}
+  CUtensorMap qp;         // absorbed query {576, 128, rows}, box {64, 1, 128} (q_pe at 512)
+  CUtensorMap kvb;        // rebuilt keys / values {H*256, keys, B}, box {64, 128, 1}
+  CUtensorMap pe;         // rotary cache {64, L, B},          box {64, 128, 1}
+};
+cudaError_t fmha_prepare();
+cudaError_t launch_fmha(const FmhaMaps& m, const FmhaParams& p, cudaStream_t s, bool pdl);
 
 // ---------------------------------------------------------------------------------------
 // a5–a7: latent flash attention (cluster of two CTAs splits the 576-wide contraction and the
@@ -107,6 +155,12 @@ struct AttnParams {
   float* part_lse;              // [pairs, 2, 128]
   const int* pair_row;          // [pairs] first row of each pair's key range, or null
   int* status;
+  unsigned long long wait_limit_ns;   // bound of every wait in the kernel (0: the 2 s default)
+  // index-mask decode (null: dense): key j of row r is cache row topk_idx[r * topk_k + j] of its
+  // sequence, gathered through the 2-D maps kv2 / pe2 (row = b * seq_rows + index)
+  const int32_t* topk_idx;
+  int topk_k;
+  long long seq_rows;           // cache rows per sequence in the 2-D view (batch stride / row stride)
 };
 
 struct CombineParams {
@@ -150,24 +204,33 @@ struct LaunchCfg {
 // Launchers (defined next to their kernels).  pdl: see LaunchCfg.
 cudaError_t launch_rmsnorm(const RmsParams& p, cudaStream_t s);
 cudaError_t launch_key_prefix(const RmsParams& p, cudaStream_t s);   // row_prefix only
+cudaError_t launch_kv_finish(const KvFinishParams& p, cudaStream_t s, bool pdl);
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                         int batches, cudaStream_t s, bool pdl);
-// Tensor maps of the attention kernel, built on the host for each call (all 128-byte swizzle).
+// Tensor maps of the attention kernel, built on the host for each call.
 struct AttnMaps {
-  CUtensorMap kv;    // latent cache  bf16 {512, max_seq_len, batch}, box {64, 32, 1}
-  CUtensorMap pe;    // rotary cache  bf16 {64, max_seq_len, batch},  box {64, 32, 1}
-  CUtensorMap q;     // absorbed queries bf16 {576, 128, rows},       box {64, 128, 1}
-  CUtensorMap o;     // o_lat         bf16 {512, n_heads, rows},      box {64, 32, 1}
-  CUtensorMap part;  // split partials fp16 {512, pairs * 2 * 128},   box {64, 32}
+  CUtensorMap kv;    // latent cache  bf16 {512, max_seq_len, batch}, box {64, 64, 1}, 128-B swizzle
+  CUtensorMap pe;    // rotary cache  bf16 {64, max_seq_len, batch},  box {32, 64, 1}, 64-B swizzle
+  CUtensorMap q;     // absorbed queries bf16 {576, 128, rows},       box {64, 128, 1}, 128-B swizzle
+  CUtensorMap qpe;   // the same tensor,                              box {32, 128, 1}, 64-B swizzle
+  // index-mask decode only: the caches as 2-D row arrays for tile::gather4 (one-row boxes)
+  CUtensorMap kv2;   // bf16 {512, batch * seq_rows}, box {64, 1}, 128-B swizzle
+  CUtensorMap pe2;   // bf16 {64, batch * seq_rows},  box {32, 1}, 64-B swizzle
 };
+// The 2-D gather maps (kv2, pe2) for the index-mask decode; needs batch strides that are whole
+// multiples of the row strides.
+bool make_gather_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,
+                      int64_t pe_sb, int64_t pe_st, int batch);
 // Strides in elements; false if a map cannot be encoded (alignment, sizes).
 bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,
                          int64_t pe_sb, int64_t pe_st, int batch, int max_seq_len, const void* qabs,
-                         int rows, const void* o_lat, int n_heads, const void* part_o, int pairs);
+                         int rows);
 cudaError_t launch_attention(const AttnMaps& m, const AttnParams& p, int n_pairs, cudaStream_t s,
                              bool pdl);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s, bool pdl);
 cudaError_t launch_transpose_uk(const bf16* wkv_b, bf16* w_ukt, int n_heads, cudaStream_t s);
+cudaError_t launch_transpose_uk_fp8(const uint8_t* wkv_b, uint8_t* w_ukt, int n_heads,
+                                    cudaStream_t s);
 cudaError_t gemm_prepare();        // one-time per-device attribute set-up
 cudaError_t attention_prepare();
 

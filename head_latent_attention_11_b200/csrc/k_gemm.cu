@@ -23,6 +23,8 @@
 //               tokens at a time through shared memory and store bf16 as 16-byte vectors (8
 //               consecutive rows of one token), hand the accumulator back — overlapping the next
 //               unit's MMAs.
+#include <cuda_fp8.h>
+
 #include "internal.h"
 #include "tc100.cuh"
 
@@ -32,8 +34,12 @@ namespace {
 
 constexpr int kEpiWarps = 8;                            // two per TMEM lane quadrant
 constexpr int kEpiThreads = 32 * kEpiWarps;
-constexpr int kGemmThreads = 64 + kEpiThreads;
+constexpr int kConvThreads = 128;                       // FP8: four converter warps
 constexpr int kSlabA = 128 * 64 * 2;   // 16 KB
+constexpr int kSlabA8 = 128 * 64;      // 8 KB: an FP8 weight slab (64-byte rows, no swizzle)
+
+template <bool FP8>
+constexpr int gemm_threads() { return 64 + kEpiThreads + (FP8 ? kConvThreads : 0); }
 
 template <int BN>
 struct GemmTile {
@@ -49,11 +55,30 @@ constexpr int kMergeSlabs = kC / 64;
 // 1 KB staging block so that the global writes are 16-byte vectors.
 constexpr int kEpiStageBytes = kEpiWarps * 32 * 16 * 2;
 
-template <int BN, int STAGES, bool MERGE = false>
+template <int BN, int STAGES, bool MERGE = false, bool FP8 = false>
 constexpr int gemm_smem_bytes() {
   return 1024 /*align slack*/ + STAGES * kSlabA +
          (MERGE ? kMergeSlabs * GemmTile<BN>::kSlabB : STAGES * GemmTile<BN>::kSlabB) +
-         256 /*barriers*/ + kEpiStageBytes;
+         (FP8 ? STAGES * kSlabA8 : 0) + 512 /*barriers*/ + kEpiStageBytes;
+}
+
+// 16 FP8 E4M3 codes (bytes of v, lowest first) times `scale` → 16 bf16 (lo: codes 0-7).
+// E4M3 values are exact in fp16 and fp32; the scaled value is rounded to fp32, then to bf16.
+__device__ __forceinline__ void fp8x16_to_bf16(const uint4 v, float scale, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 h0(__nv_cvt_fp8x2_to_halfraw2(
+        static_cast<__nv_fp8x2_storage_t>(w[i] & 0xFFFFu), __NV_E4M3));
+    const __half2 h1(__nv_cvt_fp8x2_to_halfraw2(
+        static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3));
+    const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+    o[2 * i] = pack_bf16x2(f0.x * scale, f0.y * scale);
+    o[2 * i + 1] = pack_bf16x2(f1.x * scale, f1.y * scale);
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 // Builds B = o_lat[n0 .. n0+BN)[g][0..512) (bf16, K-major, 128-byte swizzle, 8 slabs of BN rows x
@@ -279,35 +304,39 @@ struct Sched {
   }
 };
 
-template <int BN, int STAGES, bool MERGE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+template <int BN, int STAGES, bool MERGE, bool FP8>
+__global__ void __launch_bounds__(gemm_threads<FP8>(), 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmParams p, const int batches) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;
+  uint8_t* sA = smem;                      // bf16 weight slabs (FP8: written by the converters)
   uint8_t* sB = smem + STAGES * kSlabA;   // MERGE: the tile's 8 B slabs; else the ring's B slabs
   constexpr int kSmemB = MERGE ? kMergeSlabs * GemmTile<BN>::kSlabB : STAGES * GemmTile<BN>::kSlabB;
-  constexpr uint32_t kStageTx = MERGE ? kSlabA : kSlabA + GemmTile<BN>::kSlabB;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kSmemB);
+  uint8_t* sA8 = sB + kSmemB;              // FP8: the ring's fp8 weight slabs
+  constexpr uint32_t kStageTx =
+      (FP8 ? kSlabA8 : kSlabA) + (MERGE ? 0 : GemmTile<BN>::kSlabB);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sA8 + (FP8 ? STAGES * kSlabA8 : 0));
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;        // [2]
   uint64_t* acc_empty = bars + 2 * STAGES + 2;   // [2]
   uint64_t* drain = bars + 2 * STAGES + 4;
   uint64_t* b_ready = bars + 2 * STAGES + 5;     // MERGE: the tile's B block is built
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
+  uint64_t* conv = bars + 2 * STAGES + 6;        // FP8: [STAGES] the slab is converted
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint8_t* sEpi = reinterpret_cast<uint8_t*>(bars) + 256;   // plain-store epilogue staging
+  uint8_t* sEpi = reinterpret_cast<uint8_t*>(bars) + 512;   // plain-store epilogue staging
+  static_assert((3 * 10 + 6) * 8 + 8 <= 512, "barrier block");
 
   pdl_launch_dependents();
   const int warp = warp_id();
   const int nk = p.K / 64;
-  const int mt = p.M / 128;
+  const int mt = (p.M + 127) / 128;   // a last partial tile reads zero rows (TMA fill)
   const int nt = (p.N + BN - 1) / BN;
   const int total = batches * mt * nt;
-  Guard guard{abort_flag, p.status};
+  Guard guard{abort_flag, p.status, p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs};
   Sched sched;
   sched.init(total, gridDim.x, blockIdx.x);
 
@@ -322,6 +351,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(drain, 1);
     mbar_init(b_ready, kEpiThreads);
+    if (FP8)
+      for (int i = 0; i < STAGES; ++i) mbar_init(&conv[i], kConvThreads);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -346,8 +377,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const Unit un = unit_of(u, mt, nt, BN);
           for (int j = 0; j < nk && npre < STAGES; ++j, ++npre) {
             mbar_arrive_expect_tx(&full[npre], kStageTx);
-            tma_load_3d_hint(sA + npre * kSlabA, &tmA, &full[npre], j * 64, un.m0 + p.a_row_off,
-                             un.g, pol_w);
+            tma_load_3d_hint(FP8 ? sA8 + npre * kSlabA8 : sA + npre * kSlabA, &tmA, &full[npre],
+                             j * 64, un.m0 + p.a_row_off, un.g, pol_w);
           }
         }
       }
@@ -365,10 +396,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(&full[s], kStageTx);
-            tma_load_3d_hint(sA + s * kSlabA, &tmA, &full[s], j * 64, un.m0 + p.a_row_off, un.g,
-                             pol_w);
+            tma_load_3d_hint(FP8 ? sA8 + s * kSlabA8 : sA + s * kSlabA, &tmA, &full[s], j * 64,
+                             un.m0 + p.a_row_off, un.g, pol_w);
           }
-          if (!MERGE) tma_load_3d(sB + s * GemmTile<BN>::kSlabB, &tmB, &full[s], j * 64, un.g, un.n0);
+          if (!MERGE)
+            tma_load_3d(sB + s * GemmTile<BN>::kSlabB, &tmB, &full[s], j * 64, p.b_g0 ? 0 : un.g,
+                        un.n0);
         }
       }
       if (guard.aborted()) {
@@ -393,7 +426,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t d = tmem + ab * BN;
         for (int j = 0; j < nk; ++j, ++ks) {
           const int s = ks % STAGES;
-          if (!mbar_wait(&full[s], (ks / STAGES) & 1, guard)) { ok = false; break; }
+          if (!mbar_wait(FP8 ? &conv[s] : &full[s], (ks / STAGES) & 1, guard)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * kSlabA);
           const uint32_t b0 = smem_u32(sB + (MERGE ? j : s) * GemmTile<BN>::kSlabB);
@@ -409,6 +442,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ++si;
       }
       umma_commit(drain);
+    }
+  } else if (FP8 && warp >= 2 + kEpiWarps) {
+    // FP8 converter warps: each ring slab of fp8 weight codes → bf16 (code × the block's scale)
+    // in the 128-byte-swizzled layout the MMA reads; thread t converts 16-byte chunks t, t+128,
+    // t+256, t+384 of the slab (row = chunk / 4, 16 columns each)
+    const int ctid = static_cast<int>(threadIdx.x) - (64 + kEpiThreads);
+    int ks = 0;
+    int u;
+    bool ok = true;
+    while (ok && sched.next(u)) {
+      const Unit un = unit_of(u, mt, nt, BN);
+      const float* sc = p.a_scale + un.g * p.a_sg + ((un.m0 + p.a_row_off) >> 7) * p.a_sm;
+      for (int j = 0; j < nk; ++j, ++ks) {
+        const int s = ks % STAGES;
+        const float scale = __ldg(sc + ((j * 64) >> 7) * p.a_sk);
+        if (!mbar_wait(&full[s], (ks / STAGES) & 1, guard)) { ok = false; break; }
+        const uint8_t* src = sA8 + s * kSlabA8;
+        uint8_t* dst = sA + s * kSlabA;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int ch = ctid + kConvThreads * q;
+          const int r = ch >> 2, c = ch & 3;
+          const uint4 v = *reinterpret_cast<const uint4*>(src + r * 64 + c * 16);
+          uint4 lo, hi;
+          fp8x16_to_bf16(v, scale, lo, hi);
+          *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * c) ^ (r & 7)) << 4)) = lo;
+          *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * c + 1) ^ (r & 7)) << 4)) = hi;
+        }
+        fence_async_smem();   // generic-proxy writes → visible to the tensor core
+        mbar_arrive(&conv[s]);
+      }
     }
   } else {
     // epilogue warps 2 .. 1+kEpiWarps → TMEM lane quadrant warp % 4
@@ -462,7 +526,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int c = static_cast<int>(lane_id()) + 32 * j;   // 64 pieces of 16 bytes
           const int t = c >> 2, part = c & 3;
           const int n = un.n0 + c0 + t;
-          if (n < p.N)
+          if (n < p.N && mw + part * 8 < p.M)   // M is a multiple of 8: whole groups only
             *reinterpret_cast<uint4*>(epi_dst8(p, un.g, mw + part * 8, n)) =
                 *reinterpret_cast<const uint4*>(stg + t * 32 + part * 8);
         }
@@ -487,7 +551,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 int g_num_sms = 0;
 
-template <int BN, int STAGES, bool MERGE>
+template <int BN, int STAGES, bool MERGE, bool FP8 = false>
 cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                           int batches, cudaStream_t s, bool pdl) {
   if (g_num_sms == 0) {
@@ -496,18 +560,19 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Ge
     cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (g_num_sms <= 0) g_num_sms = 1;
   }
-  const int total = batches * (p.M / 128) * ((p.N + BN - 1) / BN);
+  const int total = batches * ((p.M + 127) / 128) * ((p.N + BN - 1) / BN);
   const int grid = total < g_num_sms ? total : g_num_sms;
-  LaunchCfg lc(dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<BN, STAGES, MERGE>(), s, pdl);
-  return cudaLaunchKernelEx(&lc.cfg, gemm_bf16_kernel<BN, STAGES, MERGE>, ta, tb, p, batches);
+  LaunchCfg lc(dim3(grid), dim3(gemm_threads<FP8>()), gemm_smem_bytes<BN, STAGES, MERGE, FP8>(), s,
+               pdl);
+  return cudaLaunchKernelEx(&lc.cfg, gemm_bf16_kernel<BN, STAGES, MERGE, FP8>, ta, tb, p, batches);
 }
 
-template <int BN, int STAGES, bool MERGE>
+template <int BN, int STAGES, bool MERGE, bool FP8 = false>
 cudaError_t set_attr() {
-  static_assert(gemm_smem_bytes<BN, STAGES, MERGE>() <= 232448, "shared memory budget");
-  return cudaFuncSetAttribute(gemm_bf16_kernel<BN, STAGES, MERGE>,
+  static_assert(gemm_smem_bytes<BN, STAGES, MERGE, FP8>() <= 232448, "shared memory budget");
+  return cudaFuncSetAttribute(gemm_bf16_kernel<BN, STAGES, MERGE, FP8>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              gemm_smem_bytes<BN, STAGES, MERGE>());
+                              gemm_smem_bytes<BN, STAGES, MERGE, FP8>());
 }
 
 }  // namespace
@@ -516,6 +581,17 @@ cudaError_t set_attr() {
 // The merge mode (W_UV for at most 64 rows) keeps 8 B slabs resident and a 10/8-stage A ring.
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                         int batches, cudaStream_t s, bool pdl) {
+  if (p.a_scale) {   // FP8 weights: an 8 KB fp8 slab per stage on top of the bf16 one
+    if (p.bmerge) {
+      if (p.K != kC || p.N > 64) return cudaErrorInvalidValue;
+      if (p.N <= 32) return launch_gemm_t<32, 7, true, true>(ta, tb, p, batches, s, pdl);
+      return launch_gemm_t<64, 6, true, true>(ta, tb, p, batches, s, pdl);
+    }
+    if (p.N <= 32) return launch_gemm_t<32, 7, false, true>(ta, tb, p, batches, s, pdl);
+    if (p.N <= 64) return launch_gemm_t<64, 6, false, true>(ta, tb, p, batches, s, pdl);
+    if (p.N <= 128) return launch_gemm_t<128, 5, false, true>(ta, tb, p, batches, s, pdl);
+    return launch_gemm_t<256, 3, false, true>(ta, tb, p, batches, s, pdl);
+  }
   if (p.bmerge) {
     if (p.K != kC || p.N > 64) return cudaErrorInvalidValue;
     if (p.N <= 32) return launch_gemm_t<32, 10, true>(ta, tb, p, batches, s, pdl);
@@ -534,7 +610,13 @@ cudaError_t gemm_prepare() {
   if ((e = set_attr<128, 6, false>()) != cudaSuccess) return e;
   if ((e = set_attr<256, 4, false>()) != cudaSuccess) return e;
   if ((e = set_attr<32, 10, true>()) != cudaSuccess) return e;
-  return set_attr<64, 8, true>();
+  if ((e = set_attr<64, 8, true>()) != cudaSuccess) return e;
+  if ((e = set_attr<32, 7, false, true>()) != cudaSuccess) return e;
+  if ((e = set_attr<64, 6, false, true>()) != cudaSuccess) return e;
+  if ((e = set_attr<128, 5, false, true>()) != cudaSuccess) return e;
+  if ((e = set_attr<256, 3, false, true>()) != cudaSuccess) return e;
+  if ((e = set_attr<32, 7, true, true>()) != cudaSuccess) return e;
+  return set_attr<64, 6, true, true>();
 }
 
 // W_UK^T copy made once at set-up: w_ukt[h][c][d] = wkv_b[h*256 + d][c], d < 128, so that the
@@ -549,6 +631,27 @@ __global__ void transpose_uk_kernel(const bf16* __restrict__ wkv_b, bf16* __rest
   __syncthreads();
   for (int i = ty; i < 32; i += 8)
     w_ukt[(static_cast<size_t>(h) * kC + c0 + i) * kDn + d0 + tx] = tile[tx][i];
+}
+
+// FP8 codes of W_UK^T: w_ukt[h][c][d] = wkv_b[h*256 + d][c] (bytes), d < 128.
+__global__ void transpose_uk_fp8_kernel(const uint8_t* __restrict__ wkv_b,
+                                        uint8_t* __restrict__ w_ukt) {
+  __shared__ uint8_t tile[32][33];
+  const int h = blockIdx.z;
+  const int c0 = blockIdx.x * 32, d0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
+  for (int i = ty; i < 32; i += 8)
+    tile[i][tx] = wkv_b[(static_cast<size_t>(h) * (kDn + kDv) + d0 + i) * kC + c0 + tx];
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8)
+    w_ukt[(static_cast<size_t>(h) * kC + c0 + i) * kDn + d0 + tx] = tile[tx][i];
+}
+
+cudaError_t launch_transpose_uk_fp8(const uint8_t* wkv_b, uint8_t* w_ukt, int n_heads,
+                                    cudaStream_t s) {
+  dim3 grid(kC / 32, kDn / 32, n_heads), block(32, 8);
+  transpose_uk_fp8_kernel<<<grid, block, 0, s>>>(wkv_b, w_ukt);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_transpose_uk(const bf16* wkv_b, bf16* w_ukt, int n_heads, cudaStream_t s) {

@@ -30,6 +30,20 @@ __device__ __forceinline__ int row_position(const RmsParams& p, int row, bool* b
   return pos;
 }
 
+// Keys a row attends: every key 0..position (dense), or the row's count of selected keys
+// (index-mask decode), clamped to [1, min(K, position + 1)] with the clamp reported.
+__device__ __forceinline__ int row_keys(const RmsParams& p, int row, bool* bad) {
+  const int pos = row_position(p, row, bad);
+  if (!p.topk_len) return pos + 1;
+  int n = p.topk_len[row];
+  const int cap = pos + 1 < p.topk_k ? pos + 1 : p.topk_k;
+  if (n < 1 || n > cap) {
+    *bad = true;
+    n = n < 1 ? 1 : cap;
+  }
+  return n;
+}
+
 __device__ void key_prefix_block(const RmsParams& p) {
   // 128 threads; thread t owns rows [t*chunk, (t+1)*chunk).  Block-wide scan of the per-thread
   // key counts (warp shuffles, then the four warp totals), then each thread writes its rows'
@@ -40,7 +54,7 @@ __device__ void key_prefix_block(const RmsParams& p) {
   const int r0 = min(p.rows, t * chunk), r1 = min(p.rows, r0 + chunk);
   long long local = 0;
   bool bad = false;
-  for (int r = r0; r < r1; ++r) local += row_position(p, r, &bad) + 1;
+  for (int r = r0; r < r1; ++r) local += row_keys(p, r, &bad);
   long long incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -65,7 +79,7 @@ __device__ void key_prefix_block(const RmsParams& p) {
   };
   for (int r = r0; r < r1; ++r) {
     const long long R0 = acc;
-    acc += row_position(p, r, &bad) + 1;
+    acc += row_keys(p, r, &bad);
     p.row_prefix[r + 1] = acc;
     if (p.pair_row) {
       const long long qa = first_pair_at(R0), qb = first_pair_at(acc);
@@ -194,6 +208,69 @@ cudaError_t launch_rmsnorm(const RmsParams& p, cudaStream_t s) {
       return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
+// Cache producer, second half: the wkv_a output c = [latent (512) ‖ rotary key (64)] of each new
+// token → kv_cache row = RMSNorm(latent) with the kv_norm gain, pe_cache row = RoPE(key) at the
+// token's position ("Query heads" mla-init: kv_norm = RMSNorm(kv_lora_rank); "Kimi-K2 ·
+// value_states" mla-init: the joint down-projection also emits the shared rotary key).
+// One warp per row: lane l holds latent columns 16l .. 16l+15 and rotary pair l.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) kv_finish_kernel(const KvFinishParams p) {
+  pdl_launch_dependents();
+  pdl_wait();   // c comes from the wkv_a GEMM
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 4 + warp;
+  if (row >= p.rows) return;
+  const int b = row / p.T, t = row - b * p.T;
+  const long long pos = static_cast<long long>(p.start_pos_dev ? p.start_pos_dev[b] : p.start_pos) + t;
+  if (pos < 0 || pos >= p.max_seq_len) {   // recorded, nothing written
+    if (lane == 0) atomicCAS(p.status, kDevOk, kDevBadArg);
+    return;
+  }
+  const bf16* c = p.c + static_cast<size_t>(row) * kDk;
+  const uint4* c4 = reinterpret_cast<const uint4*>(c);
+  const uint4 a0 = c4[2 * lane], a1 = c4[2 * lane + 1];
+  const __nv_bfloat162 kp = reinterpret_cast<const __nv_bfloat162*>(c + kC)[lane];
+  const float4* g4 = reinterpret_cast<const float4*>(p.gain) + 4 * lane;
+  const float4 ga = g4[0], gb = g4[1], gc = g4[2], gd = g4[3];
+  float u[16];
+  const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(&a0);
+  const __nv_bfloat16* bb = reinterpret_cast<const __nv_bfloat16*>(&a1);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    u[i] = __bfloat162float(ab[i]);
+    u[8 + i] = __bfloat162float(bb[i]);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) ss = fmaf(u[i], u[i], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = rsqrtf(ss / static_cast<float>(kC) + p.eps);
+  const float g[16] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w,
+                       gc.x, gc.y, gc.z, gc.w, gd.x, gd.y, gd.z, gd.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    o[i] = pack_bf16x2(g[2 * i] * (u[2 * i] * inv), g[2 * i + 1] * (u[2 * i + 1] * inv));
+  uint4* kv = reinterpret_cast<uint4*>(p.kv_cache + b * p.kv_sb + pos * p.kv_st) + 2 * lane;
+  kv[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  kv[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  // rotary key: pair `lane` rotated by pos * theta^(-2 lane / 64), angle in double precision
+  const double inv_freq = exp(-2.0 * static_cast<double>(lane) / kDr * p.rope_log_theta);
+  double sn, cs;
+  sincos(static_cast<double>(pos) * inv_freq, &sn, &cs);
+  const float x0 = __low2float(kp), x1 = __high2float(kp);
+  const float fc = static_cast<float>(cs), fs = static_cast<float>(sn);
+  reinterpret_cast<uint32_t*>(p.pe_cache + b * p.pe_sb + pos * p.pe_st)[lane] =
+      pack_bf16x2(x0 * fc - x1 * fs, x0 * fs + x1 * fc);
+}
+
+cudaError_t launch_kv_finish(const KvFinishParams& p, cudaStream_t s, bool pdl) {
+  LaunchCfg lc(dim3((p.rows + 3) / 4), dim3(128), 0, s, pdl);
+  return cudaLaunchKernelEx(&lc.cfg, kv_finish_kernel, p);
 }
 
 // Cumulative key counts of decode rows only (one block); used by the no-allocation attention

@@ -96,7 +96,7 @@ extern "C" mla_status mla_latent_attention_noalloc(
   const int pairs = attention_pairs() < kNoAllocPairs ? attention_pairs() : kNoAllocPairs;
   AttnMaps am;
   if (!make_attention_maps(&am, kv_cache, kv_stride_b, kv_stride_t, pe_cache, pe_stride_b,
-                           pe_stride_t, rows, max_seq_len, q_abs, rows, o_lat, n_heads, part_o, pairs))
+                           pe_stride_t, rows, max_seq_len, q_abs, rows))
     return MLA_ERR_INVALID_ARG;
 
   // the prefix and partials in the scratch array are written before they are read within the

@@ -2,9 +2,10 @@
 // tensor-memory (TMEM) allocation and loads, tcgen05 MMA issue, shared-memory matrix descriptors
 // and the cluster (distributed shared memory) primitives the kernels use.
 //
-// Every wait in this file is bounded: after ~kWaitLimitNs of failed polling it records a status
-// in the kernel's global status word, raises the CTA's shared abort flag and returns false, so a
-// stuck pipeline ends the kernel instead of hanging the GPU.
+// Every wait in this file is bounded: after the guard's limit (kWaitLimitNs = 2 s unless the
+// launch sets another) of failed polling it records a status in the kernel's global status word,
+// raises the CTA's shared abort flag and returns false, so a stuck pipeline ends the kernel
+// instead of hanging the GPU.
 #pragma once
 
 #include <cuda.h>
@@ -58,6 +59,7 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 struct Guard {
   volatile int* abort_smem;   // CTA-local flag: set once any warp gave up
   int* status_gmem;           // kernel status word in global memory
+  unsigned long long limit_ns = kWaitLimitNs;   // how long one wait may poll before giving up
   __device__ __forceinline__ bool aborted() const { return *abort_smem != 0; }
   __device__ __forceinline__ void fail(int code) const {
     *abort_smem = 1;
@@ -123,7 +125,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     if (kClusterAcquire ? mbar_test_cluster(a, parity) : mbar_test(a, parity)) return true;
     if ((++n & 63u) == 0) {
       if (g.aborted()) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > g.limit_ns) {
         g.fail(kDevTimeout);
         return false;
       }
@@ -189,6 +191,19 @@ __device__ __forceinline__ void tma_load_3d_hint(void* smem_dst, const CUtensorM
       ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
       "l"(policy)
+      : "memory");
+}
+
+// Gather four rows (r0..r3, any order) of a 2-D tensor map whose box is one row high into four
+// consecutive box rows of shared memory (swizzled as the map says).
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* m, uint64_t* bar,
+                                            int32_t x, int32_t r0, int32_t r1, int32_t r2,
+                                            int32_t r3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3), "l"(policy)
       : "memory");
 }
 
@@ -331,6 +346,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// Same descriptor for a 64-byte-swizzled K-major operand (layout type 4): rows of 64 B (32 bf16
+// along K), 8-row groups `sbo` bytes apart (512 for dense rows).  Tiles start on 512-byte
+// boundaries; a K step of 16 elements advances the start address by 32 bytes.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1) << 16;   // LBO unused for swizzled K-major layouts
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(4) << 61;
+  return d;
+}
+
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -407,6 +435,16 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t remote_dst, uint32_t 
       ::"r"(remote_dst), "r"(local_src), "r"(bytes), "r"(remote_bar)
       : "memory");
 }
+// 16-byte store into another CTA's shared memory in the cluster; on arrival it performs
+// complete_tx(16) on the remote barrier (which lives in the same CTA as the destination).
+__device__ __forceinline__ void st_async_v4(uint32_t remote_dst, uint32_t a, uint32_t b, uint32_t c,
+                                            uint32_t d, uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(remote_dst), "r"(a), "r"(b), "r"(c), "r"(d), "r"(remote_bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -92,6 +92,20 @@ mla_status mla_init(const mla_config* cfg, const float* q_norm_gain, const void*
                     const void* wkv_b, void* workspace, size_t workspace_bytes,
                     cudaStream_t stream, mla_ctx** out);
 
+/* mla_init with FP8 E4M3 block-scaled weights ("DeepSeek-V3.2-Exp · Attention update",
+ * mla-decode: weight_dequant(wkv_b.weight, wkv_b.scale); the checkpoint stores FP8 weights with
+ * one fp32 scale per 128 x 128 block).  The weights are dequantised inside the GEMMs, block by
+ * block, to the bf16 values weight_dequant returns (code × scale, rounded to bf16), so the weight
+ * bytes streamed per call are halved.
+ *   wq_b_fp8 [H·(Dn+Dr), R] and wkv_b_fp8 [H·(Dn+Dv), C]: one E4M3 code per byte, same layouts
+ *   as mla_init's bf16 weights; wq_b_scale [H·(Dn+Dr)/128, R/128] fp32 and wkv_b_scale
+ *   [H·(Dn+Dv)/128, C/128] fp32: the scale of block (i/128, j/128).  Device pointers, borrowed.
+ * Everything else (arguments, workspace, the calls that follow) as mla_init. */
+mla_status mla_init_fp8(const mla_config* cfg, const float* q_norm_gain, const void* wq_b_fp8,
+                        const float* wq_b_scale, const void* wkv_b_fp8, const float* wkv_b_scale,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                        mla_ctx** out);
+
 void mla_destroy(mla_ctx* ctx);
 
 /* a1 alone: y = RMSNorm(x (+ residual)) over rows of length `dim`.
@@ -127,6 +141,26 @@ mla_status mla_decode(mla_ctx* ctx, const void* q_latent, void* residual, const 
                       const void* pe_cache, int64_t pe_stride_b, int64_t pe_stride_t, int32_t B,
                       void* out, float* lse, float* logits, cudaStream_t stream);
 
+/* Absorbed decode with the index mask of the V3.2 excerpt ("DeepSeek-V3.2-Exp · Attention
+ * update", mla-decode: scores += full(-inf).scatter_(-1, topk_indices, 0); the selected keys come
+ * from the caller, e.g. an indexer's top-k, "DeepSeek-V3.2-Exp · Indexer":
+ * topk = min(index_topk, end_pos)).  Sequence b attends only keys topk_idx[b*k + j],
+ * j < topk_len[b]; everything else is as mla_decode (the query's RoPE position is start_pos[b]).
+ *   topk_idx [B, k] int32 (device): distinct key indices in [0, start_pos[b]] (a duplicate would
+ *     count its key twice; an index outside [0, rows per sequence) is reported as
+ *     MLA_ERR_DEVICE_ARG by mla_sync_status and read as key 0);
+ *   topk_len [B] int32 (device): 1 <= topk_len[b] <= min(k, start_pos[b] + 1) (clamped into that
+ *     range and reported as MLA_ERR_DEVICE_ARG otherwise).
+ * The cache rows are gathered by index (four rows per TMA operation): kv_stride_b must be a whole
+ * multiple of kv_stride_t, pe_stride_b of pe_stride_t, with the same quotient (rows per
+ * sequence), as in the packed layout.  No logits output. */
+mla_status mla_decode_sparse(mla_ctx* ctx, const void* q_latent, void* residual,
+                             const int32_t* start_pos, const int32_t* topk_idx,
+                             const int32_t* topk_len, int32_t k, const void* kv_cache,
+                             int64_t kv_stride_b, int64_t kv_stride_t, const void* pe_cache,
+                             int64_t pe_stride_b, int64_t pe_stride_t, int32_t B, void* out,
+                             float* lse, cudaStream_t stream);
+
 /* Absorbed attention for a chunk of T new tokens per sequence appended after `start_pos` cached
  * positions (causal: token t sees keys 0..start_pos+t, the additive -inf mask of the "Kimi-K2 ·
  * value_states" page's mla-prefill excerpt).  Cache rows start_pos..start_pos+T-1 must already
@@ -138,6 +172,27 @@ mla_status mla_prefill_chunk(mla_ctx* ctx, const void* q_latent, void* residual,
                              int64_t kv_stride_t, const void* pe_cache, int64_t pe_stride_b,
                              int64_t pe_stride_t, int32_t B, void* out, float* lse,
                              cudaStream_t stream);
+
+/* The prefill chunk in the non-absorbed form ("Kimi-K2 · value_states", mla-prefill: every head's
+ * key [W_UK kv ‖ k_pe] and value W_UV kv are rebuilt from the latent cache, then multi-head
+ * attention with the additive causal mask and an fp32 softmax), followed optionally by the output
+ * projection ("DeepSeek-V3.2-Exp · Attention update", mla-output: wo on the flattened heads).
+ * Same result as mla_prefill_chunk up to rounding (the two forms are associative rewrites of
+ * each other); this form does more arithmetic but no per-head absorption.
+ *   Arguments as mla_prefill_chunk, plus:
+ *   kv_scratch / scratch_bytes — device memory for the rebuilt keys and values of every head,
+ *     at least mla_mha_scratch_size(ctx, B, T, start_pos) bytes (B·(start_pos+T)·H·256 bf16),
+ *     16-byte aligned, owned by the caller (MLA_ERR_WORKSPACE if smaller);
+ *   wo [dim, H·Dv] bf16 (nn.Linear layout) or NULL; dim a multiple of 8 in [8, 65536];
+ *   y [B·T, dim] bf16 — wo applied to out (when wo is given).
+ * Contexts made by mla_init_fp8 return MLA_ERR_UNSUPPORTED. */
+size_t mla_mha_scratch_size(const mla_ctx* ctx, int32_t B, int32_t T, int32_t start_pos);
+mla_status mla_prefill_chunk_mha(mla_ctx* ctx, const void* q_latent, void* residual,
+                                 int32_t start_pos, int32_t T, const void* kv_cache,
+                                 int64_t kv_stride_b, int64_t kv_stride_t, const void* pe_cache,
+                                 int64_t pe_stride_b, int64_t pe_stride_t, int32_t B,
+                                 void* kv_scratch, size_t scratch_bytes, void* out, float* lse,
+                                 const void* wo, int32_t dim, void* y, cudaStream_t stream);
 
 /* Latent attention without allocating memory (no counterpart on the source pages; an addition
  * for callers that cannot allocate device memory where they run, e.g. code confined to a
@@ -170,6 +225,33 @@ mla_status mla_latent_attention_noalloc(const void* q_abs, const int32_t* start_
                                         int32_t max_seq_len, void* o_lat, float* lse,
                                         int32_t* status, cudaStream_t stream);
 
+/* Cache producer: the step upstream of the attention for new tokens ("DeepSeek-V3.2-Exp · Query
+ * heads", mla-init: wq_a = Linear(dim, q_lora_rank), wkv_a = Linear(dim, kv_lora_rank +
+ * qk_rope_head_dim), kv_norm = RMSNorm(kv_lora_rank); mla-queries: qr = q_norm(wq_a(x));
+ * "Kimi-K2 · value_states", mla-init: the joint key-value down-projection also emits the shared
+ * rotary key).  mla_attach_producer borrows the weights for later mla_produce calls:
+ *   wq_a [R, dim] bf16, wkv_a [C + Dr, dim] bf16 (nn.Linear layout [out, in]; the first C outputs
+ *   of wkv_a are the latent, the last Dr the rotary key), kv_norm_gain [C] fp32;
+ *   dim a multiple of 64 in [64, 65536] (MLA_ERR_UNSUPPORTED otherwise).  Device pointers,
+ *   16-byte aligned; they must outlive the context. */
+mla_status mla_attach_producer(mla_ctx* ctx, int32_t dim, const void* wq_a, const void* wkv_a,
+                               const float* kv_norm_gain);
+
+/* For B sequences with T new tokens each (row r = b*T + t):
+ *   q_latent[r] = x[r] wq_a^T  — [B*T, R] bf16 out, the input of mla_decode / mla_prefill_chunk;
+ *   c = x[r] wkv_a^T (bf16); kv_cache row of (b, pos) = RMSNorm(c[:C]) with the kv_norm gain and
+ *   the context's eps, bf16; pe_cache row of (b, pos) = interleaved RoPE of c[C:] at pos (the
+ *   context's rope_theta), bf16 — with pos = start_pos[b] + t (start_pos: [B] int32 on the
+ *   device) or start_pos_host + t when start_pos is NULL.  Cache arguments as for mla_decode;
+ *   only the new rows are written.  x [B*T, dim] bf16.  1 <= B*T <= cfg.max_rows.  A position
+ *   outside [0, max_seq_len) is not written and is reported as MLA_ERR_DEVICE_ARG by
+ *   mla_sync_status.  The rows are written in stream order before any later mla_decode /
+ *   mla_prefill_chunk on the same stream reads them (the pages write the cache, then attend). */
+mla_status mla_produce(mla_ctx* ctx, const void* x, const int32_t* start_pos, int32_t start_pos_host,
+                       int32_t T, int32_t B, void* kv_cache, int64_t kv_stride_b,
+                       int64_t kv_stride_t, void* pe_cache, int64_t pe_stride_b,
+                       int64_t pe_stride_t, void* q_latent, cudaStream_t stream);
+
 /* Synchronise `stream`, then read and clear the device status word of `ctx`: MLA_OK,
  * MLA_ERR_DEVICE_TIMEOUT or MLA_ERR_DEVICE_ARG (or MLA_ERR_CUDA if the synchronisation failed). */
 mla_status mla_sync_status(mla_ctx* ctx, cudaStream_t stream);
@@ -188,7 +270,15 @@ mla_status mla_stage_times(mla_ctx* ctx, float* ms, const char** names, int32_t 
 mla_status mla_debug_copy(mla_ctx* ctx, int32_t which, void* dst, size_t bytes,
                           cudaStream_t stream);
 
-/* Number of kernels the last decode / prefill call launched. */
+/* Test hook for the failure path: every wait inside the context's GEMM kernels (wq_b, the
+ * absorption, W_UV, the producer's projections, the key/value rebuild, wo) gives up after `ns`
+ * nanoseconds instead of 2 s (0 restores 2 s).  A wait that gives up makes the kernel record
+ * MLA_ERR_DEVICE_TIMEOUT (read by mla_sync_status), drain its copies and MMAs, release its tensor
+ * memory and return; the results of that call are then undefined, later calls are unaffected.
+ * The attention kernels keep their 2 s bound. */
+mla_status mla_set_wait_limit(mla_ctx* ctx, uint64_t ns);
+
+/* Number of kernels the last decode / prefill / produce call launched. */
 int32_t mla_last_launch_count(const mla_ctx* ctx);
 
 #ifdef __cplusplus

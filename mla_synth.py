@@ -33,9 +33,14 @@ from concurrent.futures import ThreadPoolExecutor
 import numpy as np
 
 __all__ = [
-    "MLADims", "Workload", "WORKLOADS", "workload", "make_inputs", "f32_to_bf16_bits",
-    "bf16_bits_to_f32", "bf16_bits_to_f64",
+    "MLADims", "Workload", "WORKLOADS", "workload", "make_inputs", "make_producer_inputs",
+    "make_topk", "make_fp8_weights", "make_wo",
+    "f32_to_bf16_bits", "bf16_bits_to_f32", "bf16_bits_to_f64", "MODEL_DIM",
 ]
+
+# Model width of the pages' models (the attention update is [B, 1, 7168] on the V3.2 page; the
+# Kimi-K2 hidden size is the same): the input width of the cache producer.
+MODEL_DIM = 7168
 
 
 # --------------------------------------------------------------------------------------------
@@ -200,3 +205,64 @@ def make_inputs(w: Workload, seed: int = 0, tail: str = "zero", max_t: int | Non
             fill_row(b)
     out["cache"] = cache
     return out
+
+
+def make_producer_inputs(w: Workload, seed: int = 0, dim: int = MODEL_DIM) -> dict:
+    """Inputs of the cache producer for workload ``w``'s new tokens, from their own seed stream
+    (so ``make_inputs`` is unchanged): ``x`` [B, T, dim] bf16 ~ N(0, 1); ``wq_a`` [q_lora, dim] and
+    ``wkv_a`` [kv_lora + rope, dim] bf16 ~ N(0, 1/dim) (nn.Linear [out, in]); ``kv_gain``
+    [kv_lora] fp32 ~ U(0.5, 1.5)."""
+    d = w.dims
+    s_x, s_q, s_kv, s_g = np.random.SeedSequence([seed, 0x70726F64]).spawn(4)
+    return {
+        "dim": dim,
+        "x": _normal_bf16(np.random.default_rng(s_x), (w.batch, w.tokens, dim)),
+        "wq_a": _normal_bf16(np.random.default_rng(s_q), (d.q_lora_rank, dim), dim ** -0.5),
+        "wkv_a": _normal_bf16(np.random.default_rng(s_kv), (d.cache_width, dim), dim ** -0.5),
+        "kv_gain": np.random.default_rng(s_g).uniform(0.5, 1.5, d.kv_lora_rank).astype(np.float32),
+    }
+
+
+def make_topk(start_pos: np.ndarray, k: int, seed: int = 0):
+    """A seeded stand-in for an indexer's top-k: for sequence b, min(k, start_pos[b] + 1)
+    distinct key indices drawn uniformly from [0, start_pos[b]], in random order.  Returns
+    (idx [B, k] int32 padded with -1, lengths [B] int32)."""
+    B = len(start_pos)
+    idx = np.full((B, k), -1, dtype=np.int32)
+    lens = np.empty(B, dtype=np.int32)
+    children = np.random.SeedSequence([seed, 0x746F706B]).spawn(B)
+    for b in range(B):
+        n = int(start_pos[b]) + 1
+        m = min(k, n)
+        rng = np.random.default_rng(children[b])
+        idx[b, :m] = rng.choice(n, size=m, replace=False)
+        lens[b] = m
+    return idx, lens
+
+
+def make_fp8_weights(w: Workload, seed: int = 0) -> dict:
+    """wq_b and wkv_b of workload ``w`` as a checkpoint would store them in FP8: E4M3 codes
+    (uint8, nn.Linear layout [out, in]) with one fp32 scale per 128 x 128 block.  Codes: N(0, 1)
+    draws times 16 rounded to E4M3 (torch's float8_e4m3fn conversion, round to nearest even);
+    scales U(0.75, 1.25) / (16 sqrt(fan_in)), so the dequantised weights have about the variance
+    1/fan_in of the bf16 weights."""
+    import torch
+    d = w.dims
+    out = {}
+    for tag, (name, rows, cols) in enumerate((
+            ("wq_b", d.n_heads * d.qk_head_dim, d.q_lora_rank),
+            ("wkv_b", d.n_heads * (d.qk_nope_head_dim + d.v_head_dim), d.kv_lora_rank))):
+        rng = np.random.default_rng(np.random.SeedSequence([seed, 0x66703800 + tag]))
+        v = rng.standard_normal((rows, cols), dtype=np.float32) * np.float32(16.0)
+        out[name] = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        out[name + "_scale"] = (rng.uniform(0.75, 1.25, (rows // 128, cols // 128))
+                                / (16.0 * np.sqrt(cols))).astype(np.float32)
+    return out
+
+
+def make_wo(w: Workload, seed: int = 0, dim: int = MODEL_DIM) -> np.ndarray:
+    """The output projection wo [dim, H*v] bf16 ~ N(0, 1/(H*v)) (nn.Linear [out, in])."""
+    d = w.dims
+    fan_in = d.n_heads * d.v_head_dim
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 0x776F]))
+    return _normal_bf16(rng, (dim, fan_in), fan_in ** -0.5)

@@ -22,7 +22,7 @@ def lib():
 def _declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    names = re.findall(r"\b(mla_[a-z_]+)\s*\(", text)
+    names = re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text)
     return sorted(set(names))
 
 
