@@ -9,6 +9,7 @@
 //   5. combine            LSE merge of rows cut between SM pairs
 //   6. gemm (W_UV)        a8 → out
 #include <math.h>
+#include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -212,10 +213,14 @@ struct StageClock {
 
 mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
-#define MLA_TRY(expr)                               \
-  do {                                              \
-    cudaError_t _e = (expr);                        \
-    if (_e != cudaSuccess) return MLA_ERR_CUDA;     \
+// A launch that fails is reported on stderr with the kernel's name, then MLA_ERR_CUDA returns.
+#define MLA_TRY(expr)                                                                       \
+  do {                                                                                      \
+    cudaError_t _e = (expr);                                                                \
+    if (_e != cudaSuccess) {                                                                \
+      fprintf(stderr, "mla: %s failed: %s\n", #expr, cudaGetErrorString(_e));             \
+      return MLA_ERR_CUDA;                                                                  \
+    }                                                                                       \
   } while (0)
 
 // Index-mask decode: per row the selected keys (topk_idx [B, k], counts topk_len [B]).
@@ -246,7 +251,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
       !make_map(&tm_olat, c->o_lat(), kC, H, rws, kC * 2, static_cast<uint64_t>(H) * kC * 2, 64, 1,
                 bn) ||
       !make_attention_maps(&am, kv, kv_sb, kv_st, pe, pe_sb, pe_st, B, c->cfg.max_seq_len, c->qabs(),
-                           rows) ||
+                           rows, c->o_lat(), H, c->part_o(), c->n_pairs) ||
       (sp.idx && !make_gather_maps(&am, kv, kv_sb, kv_st, pe, pe_sb, pe_st, B)))
     return MLA_ERR_INVALID_ARG;
 
@@ -296,6 +301,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
     g1.a_scale = c->wq_scale;
     g1.a_sm = kR / 128;
     g1.a_sk = 1;
+    g1.a_scale_n = static_cast<long long>(H) * kDq / 128 * (kR / 128);
   }
   clk.mark("wq_b_rope");
   g1.wait_limit_ns = c->gemm_wait_ns;
@@ -318,6 +324,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
     g2.a_sg = 2 * (kC / 128);
     g2.a_sm = 1;
     g2.a_sk = 0;
+    g2.a_scale_n = static_cast<long long>(H) * 2 * (kC / 128);
   }
   clk.mark("absorb_w_uk");
   g2.wait_limit_ns = c->gemm_wait_ns;
@@ -363,6 +370,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
   cp.row_pieces = c->row_pieces();
   cp.o_lat = c->o_lat();
   cp.lse_out = lse;
+  cp.status = c->status();
   if (!merge_in_wuv) {
     clk.mark("combine");
     MLA_TRY(launch_combine(cp, s, true));
@@ -386,6 +394,7 @@ mla_status run_path(mla_ctx* c, const void* q_latent, void* residual, const int3
     g3.a_sg = 2 * (kC / 128);
     g3.a_sm = kC / 128;
     g3.a_sk = 1;
+    g3.a_scale_n = static_cast<long long>(H) * 2 * (kC / 128);
   }
   if (merge_in_wuv) {
     g3.bmerge = 1;

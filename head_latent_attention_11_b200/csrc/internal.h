@@ -21,7 +21,7 @@ constexpr int kDq = kDn + kDr;        // 192 query features per head
 constexpr int kDk = kC + kDr;         // 576-wide absorbed query / cache row
 constexpr int kHPad = 128;            // heads padded to one 128-row MMA tile
 constexpr int kRopePairs = kDr / 2;   // 32
-constexpr int kAttnKeysPerTile = 64;  // cache rows per attention tile (TMA box height)
+constexpr int kAttnKeysPerTile = 32;  // cache rows per attention tile (TMA box height)
 
 // ---------------------------------------------------------------------------------------
 // a1: RMSNorm (+ residual) with the rotary table and the per-row key prefix as side outputs
@@ -110,6 +110,7 @@ struct GemmParams {
   // a_scale[g * a_sg + ((m + a_row_off) / 128) * a_sm + (k / 128) * a_sk] (128 x 128 blocks)
   const float* a_scale;
   long long a_sg, a_sm, a_sk;
+  long long a_scale_n;     // elements of a_scale (an index at or past it is reported, not read)
   int b_g0;                // B is shared by every batch g (its batch coordinate is 0)
   unsigned long long wait_limit_ns;   // bound of every wait in the kernel (0: the 2 s default)
 };
@@ -174,6 +175,7 @@ struct CombineParams {
   const int2* row_pieces;       // [rows] see RmsParams::row_pieces
   bf16* o_lat;
   float* lse_out;
+  int* status;
 };
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no interleave, L2 256-byte
@@ -207,24 +209,25 @@ cudaError_t launch_key_prefix(const RmsParams& p, cudaStream_t s);   // row_pref
 cudaError_t launch_kv_finish(const KvFinishParams& p, cudaStream_t s, bool pdl);
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                         int batches, cudaStream_t s, bool pdl);
-// Tensor maps of the attention kernel, built on the host for each call.
+// Tensor maps of the attention kernel, built on the host for each call (all 128-byte swizzle).
 struct AttnMaps {
-  CUtensorMap kv;    // latent cache  bf16 {512, max_seq_len, batch}, box {64, 64, 1}, 128-B swizzle
-  CUtensorMap pe;    // rotary cache  bf16 {64, max_seq_len, batch},  box {32, 64, 1}, 64-B swizzle
-  CUtensorMap q;     // absorbed queries bf16 {576, 128, rows},       box {64, 128, 1}, 128-B swizzle
-  CUtensorMap qpe;   // the same tensor,                              box {32, 128, 1}, 64-B swizzle
+  CUtensorMap kv;    // latent cache  bf16 {512, max_seq_len, batch}, box {64, 32, 1}
+  CUtensorMap pe;    // rotary cache  bf16 {64, max_seq_len, batch},  box {64, 32, 1}
+  CUtensorMap q;     // absorbed queries bf16 {576, 128, rows},       box {64, 128, 1}
+  CUtensorMap o;     // o_lat         bf16 {512, n_heads, rows},      box {64, 32, 1}
+  CUtensorMap part;  // split partials fp16 {512, pairs * 2 * 128},   box {64, 32}
   // index-mask decode only: the caches as 2-D row arrays for tile::gather4 (one-row boxes)
-  CUtensorMap kv2;   // bf16 {512, batch * seq_rows}, box {64, 1}, 128-B swizzle
-  CUtensorMap pe2;   // bf16 {64, batch * seq_rows},  box {32, 1}, 64-B swizzle
+  CUtensorMap kv2;   // bf16 {512, batch * seq_rows}, box {64, 1}
+  CUtensorMap pe2;   // bf16 {64, batch * seq_rows},  box {64, 1}
 };
+// Strides in elements; false if a map cannot be encoded (alignment, sizes).
+bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,
+                         int64_t pe_sb, int64_t pe_st, int batch, int max_seq_len, const void* qabs,
+                         int rows, const void* o_lat, int n_heads, const void* part_o, int pairs);
 // The 2-D gather maps (kv2, pe2) for the index-mask decode; needs batch strides that are whole
 // multiples of the row strides.
 bool make_gather_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,
                       int64_t pe_sb, int64_t pe_st, int batch);
-// Strides in elements; false if a map cannot be encoded (alignment, sizes).
-bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,
-                         int64_t pe_sb, int64_t pe_st, int batch, int max_seq_len, const void* qabs,
-                         int rows);
 cudaError_t launch_attention(const AttnMaps& m, const AttnParams& p, int n_pairs, cudaStream_t s,
                              bool pdl);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s, bool pdl);

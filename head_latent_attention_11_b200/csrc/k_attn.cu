@@ -9,36 +9,42 @@
 // Design (B200):
 //   * One query row (one token of one sequence) at a time; its heads form the MMA M dimension
 //     (128 rows; heads beyond H are zero rows), so QK^T and P·V are dense 128-row tcgen05 MMAs.
-//   * A cluster of TWO CTAs (one SM each) handles a row and splits the 576-wide cache row evenly:
-//     CTA r owns latent columns [256r, 256r + 256) and rotary columns [32r, 32r + 32), 288 columns
-//     = 36 KB per 64-key tile each, so every cache row crosses HBM once and both SMs move the same
-//     bytes and issue the same number of MMAs.  Each CTA computes a partial score tile over its
-//     columns and hands it to the peer; both then hold the full scores and run the same online
-//     softmax.  Each CTA accumulates the value half it owns, O[128 x 256] fp32 in TMEM.
-//   * Tiles are 64 keys: the score MMA is M=128, N=64 (a tcgen05.mma costs its issuing thread
-//     about as long as a 128x64x16 product takes the tensor core, so smaller N would leave the
-//     tensor pipe waiting on instruction issue).
-//   * The CTA's 256 latent query columns live in TMEM (A operand of the score MMA); its 32 rotary
-//     query columns stay in shared memory (64-byte swizzle).  The latent query reaches TMEM by TMA
-//     into two ring stages and tcgen05.cp, once per piece.  P (bf16) overwrites the score tile in
-//     TMEM and is the A operand of P·V.
-//     TMEM columns: O [0,256) | latent query [256,384) | two 64-column score/P buffers [384,512).
-//   * Score exchange: every lane stores its row's 64 partial scores straight from registers into
-//     the peer's receive slot for its warp (st.async, 16 B each, completing bytes on the peer
-//     warp's barrier); the peer adds them to its own partial.  No staging buffer.
-//   * Two softmax groups of four warps take tiles in turn; within a group one thread owns one head
-//     row.  Only the running-max decision is handed from tile to tile across the groups (per-row
-//     flag in shared memory); each group keeps its own partial row sum.
+//   * A cluster of TWO CTAs (one SM each) handles a row.  CTA 0 owns the latent columns
+//     [0, 256); CTA 1 owns [256, 512) and the 64 rotary columns.  Each CTA streams only its
+//     columns of every cache tile (the 576-wide cache row crosses HBM once), computes a partial
+//     score tile over them and hands it to the peer; both CTAs then hold identical full scores
+//     and run the identical online softmax.  Each CTA accumulates the value half it owns,
+//     O[128 x 256] fp32 in TMEM.
+//   * The CTA's 256 latent query columns live in TMEM (A operand of the score MMA); rank 1's 64
+//     rotary query columns stay in shared memory (A from a smem descriptor for those K-steps), so
+//     both CTAs have room for four score buffers.  The query reaches TMEM by TMA into ring slots
+//     and tcgen05.cp, once per piece.  The probabilities P (bf16) overwrite the score tile in
+//     TMEM and are the A operand of P·V.  Shared memory holds the cache ring (32-key tiles, 7
+//     stages, TMA with 128-byte swizzle, evict-first) and the exchange buffers.
+//     TMEM columns: O [0,256) | latent query [256,384) | four 32-column score/P buffers [384,512).
+//     With four buffers the score MMA of tile g only waits for P·V of tile g-4 to be issued.
+//   * Score exchange: each warp stages its 32 rows of partial scores and ships them with one
+//     4 KB bulk copy (shared::cta → the peer's receive slot), which completes a transaction count
+//     on the peer warp's own barrier; a warp waits only for its counterpart (same group and lane
+//     quarter) in the peer CTA.  The four warps of a lane quarter share one staging slot, handed
+//     from use to use in a fixed order.
+//   * Twelve softmax warps in three groups of four take turns by tile; within a group one thread
+//     owns one head row.  Only the running-max decision is handed from tile to tile across the
+//     groups (per-row flag in shared memory); each group keeps its own partial row sum, so the
+//     softmax work of consecutive tiles overlaps.
 //   * The flattened key range of all rows is split evenly over the cluster pairs (split-K over
-//     keys, also across row boundaries); a row cut between pairs leaves normalised fp16 partials
-//     (O/l) and its lse for the merge, an uncut row is written as bf16 o_lat directly, both stored
-//     from registers by the softmax threads.
+//     keys, also across row boundaries); a row cut between pairs leaves normalised partials
+//     (O/l, lse) for the combine kernel, an uncut row is written as bf16 o_lat directly, both
+//     by TMA tile stores from a swizzled staging block.
 //   * Online softmax in exp2 domain with lazy rescaling: the running max is only raised (and O
-//     in TMEM rescaled) when a tile's max exceeds it by more than 8 (factor 256).
-//   * Warp roles: warp 0 TMA producer (lane 0 dense, lanes 0-15 gathering in the index-mask mode;
-//     lane 1 or 31: the rotary query columns), warp 1 TMEM owner +
-//     score-MMA issuer (and the query copies), warp 2 P·V issuer, warps 3-10 softmax and
-//     epilogue (thread = head row = TMEM lane).
+//     in TMEM rescaled) when a tile's max exceeds it by more than 8 (factor 256), which keeps the
+//     rescale off the common path while the result stays exact.
+//   * Warp roles: warp 0 TMA producer (lane 1 of rank 1: rotary query slab; in the index-mask mode
+//     lanes 0-7 gather the cache rows by index and lane 31 loads the rotary slab), warp 1 TMEM owner
+//     + score-MMA issuer (and the query copies), warp 2 P·V issuer, warps 3-14 softmax and
+//     epilogue (thread = head row = TMEM lane).  A tcgen05 instruction costs a single issuing
+//     thread ~48 cycles, so the score and P·V streams are issued by two threads in parallel.
+//     The score buffer a QK reuses is handed back by the P·V thread's completion barrier.
 //   * Every wait is bounded (see tc100.cuh); a stuck pipeline records a status and ends.
 #include "internal.h"
 #include "tc100.cuh"
@@ -47,33 +53,39 @@ namespace mla {
 
 namespace {
 
-constexpr int kNK = kAttnKeysPerTile;      // 64 keys per tile
-constexpr int kStages = 4;                 // cache tile ring depth
-constexpr int kL2Ahead = 6;                // tiles the L2 look-ahead runs ahead of the ring loads
-constexpr int kL2Every = 2;                // one tile in kL2Every is prefetched into L2
-constexpr int kSlabKV = kNK * 128;         // 8 KB: 64 latent columns x 64 keys (128-byte rows)
-constexpr int kSlabPe = kNK * 64;          // 4 KB: 32 rotary columns x 64 keys (64-byte rows)
-constexpr int kStageBytes = 4 * kSlabKV + kSlabPe;   // 36 KB
-constexpr int kSlabQ = 128 * 64 * 2;       // 16 KB: 64 latent query columns of the 128 head rows
-constexpr int kSlabQPe = 128 * 32 * 2;     // 8 KB: 32 rotary query columns of the 128 head rows
-constexpr int kQStages = 2;                // ring stages carrying a piece's latent query
-constexpr int kGroups = 2;                 // softmax groups (4 warps each) taking turns by tile
-constexpr int kXWarp = 32 * kNK * 4;       // 8 KB: one warp's 32 rows of a partial score tile
+constexpr int kNK = kAttnKeysPerTile;      // keys per tile
+constexpr int kStages = 7;                 // cache tile ring depth
+// L2 look-ahead (build-time tuning): tiles it runs ahead of the ring loads, and one tile in
+// kL2Every is prefetched (0: no look-ahead)
+#ifndef MLA_ATTN_L2_AHEAD
+#define MLA_ATTN_L2_AHEAD 12
+#endif
+#ifndef MLA_ATTN_L2_EVERY
+#define MLA_ATTN_L2_EVERY 3
+#endif
+constexpr int kL2Ahead = MLA_ATTN_L2_AHEAD;
+constexpr int kL2Every = MLA_ATTN_L2_EVERY;
+constexpr int kSlabKV = kNK * 128;         // 4 KB: 64 columns x 32 keys, bf16
+constexpr int kMaxSlabs = 5;               // rank 1: 4 latent slabs + 1 rotary slab
+constexpr int kSlabQ = 128 * 64 * 2;       // 16 KB: 64 query columns of all 128 head rows
+constexpr int kStageBytes = kMaxSlabs * kSlabKV;
+constexpr int kGroups = 3;                 // softmax groups (4 warps each) taking turns by tile
+constexpr int kXWarp = 32 * kNK * 4;       // 4 KB: one warp's 32 rows of a partial score tile
 
 constexpr int kOffKV = 0;
-constexpr int kOffX = kOffKV + kStages * kStageBytes;   // receive slots [group][lane quarter]
-constexpr int kOffQPe = kOffX + kGroups * 4 * kXWarp;   // the piece's rotary query columns
-constexpr int kOffRed = kOffQPe + kSlabQPe;             // m_ref, seq, row sums
-constexpr int kRedBytes = (2 + 2 * kGroups) * 128 * 4;
-constexpr int kOffBar = kOffRed + kRedBytes;
-constexpr int kAttnSmem = kOffBar + 512 + 1024;         // barriers + alignment slack
+constexpr int kOffX = kOffKV + kStages * kStageBytes;     // receive slots (peer → this CTA), per warp
+constexpr int kOffY = kOffX + kGroups * 4 * kXWarp;       // staging slots, one per lane quarter
+constexpr int kOffQPe = kOffY + 4 * kXWarp;               // rank 1: rotary query slab (A from smem)
+constexpr int kOffRed = kOffQPe + kSlabQ;                 // row-max / row-sum exchange
+constexpr int kOffBar = kOffRed + (2 + 2 * kGroups) * 128 * 4;
+constexpr int kAttnSmem = kOffBar + 768 + 1024;
 
 constexpr int kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;             // [0, 256)
 constexpr uint32_t kTmemQ = 256;           // [256, 384): 256 bf16 latent query columns
-constexpr uint32_t kTmemS = 384;           // two 64-column score / probability buffers
-constexpr int kNS = 2;
-constexpr int kNB = 4;                     // ring of per-tile barrier slots (s_full, pv_done)
+constexpr uint32_t kTmemS = 384;           // four 32-column score / probability buffers
+constexpr int kNS = 4;
+constexpr int kNB = 8;                     // ring of per-tile barrier slots (s_full, pv_done)
 
 constexpr int kSoftmaxWarps = 4 * kGroups;
 constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
@@ -84,38 +96,45 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_empty;         // the piece's last score MMA has read the query (TMEM and smem)
-  uint64_t qpe_full;        // the piece's rotary query columns have landed
+  uint64_t qpe_full;        // rank 1: the piece's rotary query slab has landed
   uint64_t s_full[kNB], p_full[kNS], pv_done[kNB];
   uint64_t o_empty;
-  uint64_t x_full[4 * kGroups], x_empty[4 * kGroups];   // [group][lane quarter]
+  uint64_t x_full[4 * kGroups], x_empty[4 * kGroups];   // [group][warp quad]
   uint64_t sync_all;        // all softmax threads
   uint64_t drain;
   uint32_t tmem_slot;
   int abort_flag;
+  // staging slot of each lane quarter: number of uses that have released it (a counter, not a
+  // barrier: a warp may start waiting for its turn more than one use ahead)
+  int y_released[4];
 };
-static_assert(sizeof(Bars) <= 512, "barrier block");
+static_assert(sizeof(Bars) <= 768, "barrier block");
 static_assert(kAttnSmem <= 232448, "shared memory budget");
-static_assert(kStageBytes % 1024 == 0 && kOffX % 1024 == 0 && kOffQPe % 1024 == 0,
-              "swizzled tiles start on 1024-byte boundaries");
 
 // Iterates the pieces (row, [k0, k1)) of one pair's key range.
 struct PieceIter {
   const long long* prefix;
   int rows;
   long long e0, e1;
+  long long max_keys;   // keys a row can have (cache rows per sequence)
   int r;
   // first_row: the row containing key b when known (else -1: binary search)
-  __device__ void init(const long long* pf, int nrows, long long b, long long e, int first_row) {
+  __device__ void init(const long long* pf, int nrows, long long b, long long e, int first_row,
+                       long long maxk) {
     prefix = pf;
     rows = nrows;
     e0 = b;
     e1 = e;
-    r = first_row >= 0 ? first_row : row_of_key(pf, nrows, b);
+    max_keys = maxk;
+    r = first_row >= 0 && first_row < nrows ? first_row : row_of_key(pf, nrows, b);
   }
+  // Key counts come from the key prefix (written by the RMSNorm kernel of the same call) and are
+  // read at L2 (coherent) so every role of the CTA pair sees the same pieces; a record that
+  // cannot come from a valid prefix ends the walk (and is reported by the caller's check).
   __device__ bool get(int& row, int& k0, int& k1, int& nkeys_row, bool& first_row) const {
-    if (r >= rows) return false;
-    const long long R0 = __ldg(prefix + r), R1 = __ldg(prefix + r + 1);
-    if (R0 >= e1) return false;
+    if (r < 0 || r >= rows) return false;
+    const long long R0 = __ldcg(prefix + r), R1 = __ldcg(prefix + r + 1);
+    if (R0 >= e1 || R0 < 0 || R1 < R0 || R1 - R0 > max_keys) return false;
     row = r;
     k0 = static_cast<int>((e0 > R0 ? e0 : R0) - R0);
     k1 = static_cast<int>((e1 < R1 ? e1 : R1) - R0);
@@ -126,44 +145,13 @@ struct PieceIter {
   __device__ void next() { ++r; }
 };
 
-// 32 lanes x 32 bit, 64 consecutive columns per thread, load + wait fused.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  float (&lo)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
-  float (&hi)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
-  tmem_ld32(taddr, lo);
-  tmem_ld32(taddr + 32, hi);
-}
-
-// Raw 32-bit words to TMEM (32 columns) and wait for the store.
-__device__ __forceinline__ void tmem_st32_u32(uint32_t taddr, const uint32_t (&r)[32]) {
-  const uint32_t (&lo)[16] = *reinterpret_cast<const uint32_t(*)[16]>(&r[0]);
-  const uint32_t (&hi)[16] = *reinterpret_cast<const uint32_t(*)[16]>(&r[16]);
-  tmem_st16_u32(taddr, lo);
-  tmem_st16_u32(taddr + 16, hi);
-}
-
-// Bounded spin on a per-row flag in shared memory written by another group.
-__device__ __forceinline__ bool wait_seq(volatile int* seq, int h, int want, const Guard& g) {
-  bool seen = true;
-  if (seq[h] != want) {
-    const unsigned long long t0 = globaltimer_ns();
-    uint32_t n = 0;
-    while (seq[h] != want) {
-      if ((++n & 63u) == 0 && (g.aborted() || globaltimer_ns() - t0 > g.limit_ns)) {
-        if (!g.aborted()) g.fail(kDevTimeout);
-        seen = false;
-        break;
-      }
-    }
-  }
-  return __all_sync(0xffffffffu, seen);
-}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     latent_attention_kernel(const __grid_constant__ CUtensorMap tmKV,
                             const __grid_constant__ CUtensorMap tmPE,
                             const __grid_constant__ CUtensorMap tmQ,
-                            const __grid_constant__ CUtensorMap tmQPe,
+                            const __grid_constant__ CUtensorMap tmO,
+                            const __grid_constant__ CUtensorMap tmPart,
                             const __grid_constant__ CUtensorMap tmKV2,
                             const __grid_constant__ CUtensorMap tmPE2, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -171,8 +159,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sKV = smem + kOffKV;
   uint8_t* sX = smem + kOffX;
-  uint8_t* sQPe = smem + kOffQPe;
-  float* sRed = reinterpret_cast<float*>(smem + kOffRed);   // m_ref, seq, row sums
+  uint8_t* sY = smem + kOffY;
+  float* sRed = reinterpret_cast<float*>(smem + kOffRed);   // m_ref, seq, 2 x row sums
   Bars* bar = reinterpret_cast<Bars*>(smem + kOffBar);
 
   // Programmatic dependent launch: the key prefix is final before this kernel can start (the
@@ -184,8 +172,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t peer = rank ^ 1u;
   const int pair = static_cast<int>(cluster_id_x());
   const int launched_pairs = static_cast<int>(nclusters_x());
-  const long long total = __ldg(p.row_prefix + p.rows);
-  const int row0 = p.pair_row ? __ldg(p.pair_row + pair) : -1;   // same round trip as total
+  const long long total = __ldcg(p.row_prefix + p.rows);
+  const int row0 = p.pair_row ? __ldcg(p.pair_row + pair) : -1;   // same round trip as total
   const int pairs = active_pairs(total, launched_pairs, p.min_keys_per_pair);
   if (pair >= pairs) {         // both CTAs of the pair take this branch together
     pdl_wait();
@@ -194,8 +182,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const long long e0 = pair_begin(total, pairs, pair), e1 = pair_begin(total, pairs, pair + 1);
 
   const int warp = static_cast<int>(warp_id());
-  const int col0 = static_cast<int>(rank) * 256;   // first latent column this CTA owns
-  const int pe0 = static_cast<int>(rank) * 32;     // first rotary column this CTA owns
+  const int nslabs = rank == 0 ? 4 : 5;           // 64-column cache slabs this CTA owns
+  const int col0 = rank == 0 ? 0 : 256;           // first cache / query column it owns
+  uint8_t* sQPe = smem + kOffQPe;                 // rank 1: the rotary query slab
   Guard guard{reinterpret_cast<volatile int*>(&bar->abort_flag), p.status,
               p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs};
 
@@ -212,9 +201,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kNS; ++i) mbar_init(&bar->p_full[i], 128);   // the tile's group
     for (int i = 0; i < 4 * kGroups; ++i) {
-      mbar_init(&bar->x_full[i], 1);     // the receiving warp's expect_tx + the peer's 8 KB
-      mbar_init(&bar->x_empty[i], 1);    // the peer warp has consumed this warp's last send
+      mbar_init(&bar->x_full[i], 1);     // receiving warp's expect_tx + the peer warp's 4 KB copy
+      mbar_init(&bar->x_empty[i], 1);    // the peer warp has consumed this warp's last copy
     }
+    for (int i = 0; i < 4; ++i) bar->y_released[i] = 0;
     mbar_init(&bar->o_empty, kSoftmaxThreads);
     mbar_init(&bar->sync_all, kSoftmaxThreads);
     mbar_init(&bar->drain, 2);   // both MMA-issuing threads
@@ -223,7 +213,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmKV);
     tma_prefetch_desc(&tmPE);
     tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmQPe);
+    tma_prefetch_desc(&tmO);
+    tma_prefetch_desc(&tmPart);
     if (p.topk_idx) {
       tma_prefetch_desc(&tmKV2);
       tma_prefetch_desc(&tmPE2);
@@ -237,27 +228,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bar->tmem_slot;
 
   PieceIter it;
-  it.init(p.row_prefix, p.rows, e0, e1, row0);
+  it.init(p.row_prefix, p.rows, e0, e1, row0, p.max_seq_len);
+  // The ring slot each stage was last armed for, and the rotary query slabs armed, by the thread
+  // that armed them: if any role gives up, these loads land before the CTA releases its memory.
+  int last_slot[kStages];
+  for (int s = 0; s < kStages; ++s) last_slot[s] = -1;
+  int qpe_armed = 0;
 
-  // Lane of warp 0 that loads the pieces' rotary query columns (lanes 0-15 gather in the
-  // index-mask mode).
+  // lane of warp 0 that loads rank 1's rotary query slabs (lanes 0-7 gather in the index-mask
+  // mode)
   const uint32_t qpe_lane = p.topk_idx ? 31u : 1u;
-  if (warp == 0 && p.topk_idx && lane_id() < 16) {
+  if (warp == 0 && p.topk_idx && lane_id() < 8) {
     // ---------------------------------------------------------------- TMA producer, index mask
-    // Key j of a row is cache row topk_idx[row][j] of its sequence: every tile's 64 rows are
+    // Key j of a row is cache row topk_idx[row][j] of its sequence: every tile's 32 rows are
     // gathered four at a time (tile::gather4 on the 2-D row maps, one-row boxes), lane l taking
     // keys 4l .. 4l+3 of each slab.  Slots past the piece's end load the piece's first key (a
     // valid row; its score is masked and its latent row zeroed before P·V).  Lane 0 also loads
-    // the query stages and owns the ring bookkeeping.
+    // the query slabs and owns the ring bookkeeping.
     const int lane = static_cast<int>(lane_id());
     const uint64_t pol = policy_evict_first();
     pdl_wait();
     int rs = 0;
-    int last_slot[kStages];
-    for (int s = 0; s < kStages; ++s) last_slot[s] = -1;
     int row, k0, k1, nrow;
     bool first_row;
-    bool ok = true;
+    bool ok = true, bad = false;
     auto take_slot = [&](uint32_t bytes) -> int {   // lane 0: next ring slot, armed for `bytes`
       const int s = rs % kStages;
       if (rs >= kStages && !mbar_wait(&bar->kv_empty[s], ((rs / kStages) - 1) & 1, guard))
@@ -266,21 +260,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       last_slot[s] = rs++;
       return s;
     };
-    bool bad = false;
     while (ok && it.get(row, k0, k1, nrow, first_row)) {
       const long long rowbase = static_cast<long long>(row / p.T) * p.seq_rows;
       const int32_t* idx = p.topk_idx + static_cast<size_t>(row) * p.topk_k;
       const int ntiles = (k1 - k0 + kNK - 1) / kNK;
       if (lane == 0) {
-        for (int qs = 0; qs < kQStages && ok; ++qs) {
-          const int s = take_slot(2 * kSlabQ);
+        for (int i = 0; i < 4 && ok; ++i) {
+          const int s = take_slot(kSlabQ);
           if (s < 0) { ok = false; break; }
-          for (int h = 0; h < 2; ++h)
-            tma_load_3d(sKV + s * kStageBytes + h * kSlabQ, &tmQ, &bar->kv_full[s],
-                        col0 + 64 * (2 * qs + h), 0, row);
+          tma_load_3d(sKV + s * kStageBytes, &tmQ, &bar->kv_full[s], col0 + 64 * i, 0, row);
         }
       }
-      ok = __shfl_sync(0xffffu, ok, 0);
+      ok = __shfl_sync(0xffu, ok, 0);
       int first = __ldg(idx + k0);
       if (first < 0 || first >= p.seq_rows) {
         bad = true;
@@ -302,45 +293,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           rr[i] = static_cast<int>(rowbase + t);
         }
         int s = 0;
-        if (lane == 0) s = take_slot(kStageBytes);
-        s = __shfl_sync(0xffffu, s, 0);
+        if (lane == 0) s = take_slot(nslabs * kSlabKV);
+        s = __shfl_sync(0xffu, s, 0);
         if (s < 0) { ok = false; break; }
         uint64_t* fb = &bar->kv_full[s];
         uint8_t* dst = sKV + s * kStageBytes;
         for (int i = 0; i < 4; ++i)
           tma_gather4(dst + i * kSlabKV + lane * 512, &tmKV2, fb, col0 + 64 * i, rr[0], rr[1],
                       rr[2], rr[3], pol);
-        tma_gather4(dst + 4 * kSlabKV + lane * 256, &tmPE2, fb, pe0, rr[0], rr[1], rr[2], rr[3],
-                    pol);
+        if (rank == 1)
+          tma_gather4(dst + 4 * kSlabKV + lane * 512, &tmPE2, fb, 0, rr[0], rr[1], rr[2], rr[3],
+                      pol);
       }
       it.next();
     }
     if (bad) atomicCAS(p.status, kDevOk, kDevBadArg);
-    if (lane == 0 && guard.aborted()) {
-      int dummy = 0;
-      Guard drain{reinterpret_cast<volatile int*>(&dummy), p.status};
-      for (int s = 0; s < kStages; ++s)
-        if (last_slot[s] >= 0) mbar_wait(&bar->kv_full[s], (last_slot[s] / kStages) & 1, drain);
-    }
-  } else if (warp == 0 && !p.topk_idx && lane_id() == 0) {
-    // ---------------------------------------------------------------- TMA producer, dense
-    // Lane 0: ring slot sequence per piece = two stages of latent query (two 128 x 64 slabs of
-    // 16 KB each), then the piece's cache tiles (4 latent slabs + this CTA's rotary half).
-    {
+  } else if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    // Lane 0: ring slot sequence per piece = the 4 latent query slabs this CTA owns (128 x 64
+    // columns, 16 KB each), then the piece's cache tiles.  Lane qpe_lane of rank 1: the piece's
+    // rotary query slab into its own buffer, once the previous piece's last score MMA has read it.
+    const uint32_t lane = lane_id();
+    if (lane == 0 && !p.topk_idx) {
       const uint64_t pol = policy_evict_first();
       // L2 look-ahead: a second cursor over the same tiles, kL2Ahead tiles in front of the ring
-      // loads, has the TMA unit pull one tile in kL2Every into L2, so more bytes are in flight
-      // from HBM than the ring holds.  Its first tiles go out before the wait below.  The
-      // prefetches share the TMA unit's bandwidth with the ring's loads, hence not every tile.
+      // loads, has the TMA unit pull its tiles into L2, so the bytes in flight from HBM are not
+      // limited by the ring's depth.  Its first kL2Ahead tiles go out before the wait below.
+      // Only one tile in three is prefetched: the prefetches go through the same TMA unit as the
+      // ring's loads (~48 GB/s per SM), so prefetching every tile halves the rate at which the
+      // ring can be filled; the tiles in between load from HBM within the ring's depth (every
+      // tile: 0.83 us per tile; every other: 68.5 us per launch; one in three: 67.0 us).
       PieceIter pf = it;
       bool pf_live = false, pf_done = false;
       int pf_b = 0, pf_key = 0, pf_end = 0, pf_n = 0;
       auto prefetch_next = [&]() {
         while (!pf_done) {
           if (pf_live && pf_key < pf_end) {
-            if ((pf_n++ % kL2Every) == 0) {
+            if (kL2Every > 0 && (pf_n++ % (kL2Every > 0 ? kL2Every : 1)) == 0) {
               for (int i = 0; i < 4; ++i) tma_prefetch_l2_3d(&tmKV, col0 + 64 * i, pf_key, pf_b);
-              tma_prefetch_l2_3d(&tmPE, pe0, pf_key, pf_b);
+              if (rank == 1) tma_prefetch_l2_3d(&tmPE, 0, pf_key, pf_b);
             }
             pf_key += kNK;
             return;
@@ -361,8 +352,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int i = 0; i < kL2Ahead; ++i) prefetch_next();
       pdl_wait();   // the queries come from the absorption GEMM
       int rs = 0;   // ring slot sequence number
-      int last_slot[kStages];
-      for (int s = 0; s < kStages; ++s) last_slot[s] = -1;
       int row, k0, k1, nrow;
       bool first_row;
       bool ok = true;
@@ -377,54 +366,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       while (ok && it.get(row, k0, k1, nrow, first_row)) {
         const int b = row / p.T;
         const int ntiles = (k1 - k0 + kNK - 1) / kNK;
-        for (int qs = 0; qs < kQStages && ok; ++qs) {
-          const int s = take_slot(2 * kSlabQ);
+        for (int i = 0; i < 4 && ok; ++i) {
+          const int s = take_slot(kSlabQ);
           if (s < 0) { ok = false; break; }
-          for (int h = 0; h < 2; ++h)
-            tma_load_3d(sKV + s * kStageBytes + h * kSlabQ, &tmQ, &bar->kv_full[s],
-                        col0 + 64 * (2 * qs + h), 0, row);
+          tma_load_3d(sKV + s * kStageBytes, &tmQ, &bar->kv_full[s], col0 + 64 * i, 0, row);
         }
         for (int j = 0; j < ntiles && ok; ++j) {
-          const int s = take_slot(kStageBytes);
+          const int s = take_slot(nslabs * kSlabKV);
           if (s < 0) { ok = false; break; }
           uint64_t* fb = &bar->kv_full[s];
           uint8_t* dst = sKV + s * kStageBytes;
           const int key = k0 + j * kNK;
           for (int i = 0; i < 4; ++i)
             tma_load_3d_hint(dst + i * kSlabKV, &tmKV, fb, col0 + 64 * i, key, b, pol);
-          tma_load_3d_hint(dst + 4 * kSlabKV, &tmPE, fb, pe0, key, b, pol);
+          if (rank == 1) tma_load_3d_hint(dst + 4 * kSlabKV, &tmPE, fb, 0, key, b, pol);
           prefetch_next();
         }
         it.next();
       }
-      if (guard.aborted()) {
-        int dummy = 0;
-        Guard drain{reinterpret_cast<volatile int*>(&dummy), p.status};
-        for (int s = 0; s < kStages; ++s)
-          if (last_slot[s] >= 0) mbar_wait(&bar->kv_full[s], (last_slot[s] / kStages) & 1, drain);
-      }
-    }
-  } else if (warp == 0) {
-    // ---------------------------------------------------------------- rotary query loader
-    // The piece's rotary query columns into their own buffer, once the previous piece's last
-    // score MMA has read them (lane qpe_lane; warp 0's other lanes have no role).
-    if (lane_id() == qpe_lane) {
+    } else if (lane == qpe_lane && rank == 1) {
       pdl_wait();
       int row, k0, k1, nrow, pc = 0;
       bool first_row;
-      bool armed = false;
       while (it.get(row, k0, k1, nrow, first_row)) {
         if (pc > 0 && !mbar_wait(&bar->q_empty, (pc - 1) & 1, guard)) break;
-        mbar_arrive_expect_tx(&bar->qpe_full, kSlabQPe);
-        armed = true;
-        tma_load_3d(sQPe, &tmQPe, &bar->qpe_full, kC + pe0, 0, row);
-        ++pc;
+        mbar_arrive_expect_tx(&bar->qpe_full, kSlabQ);
+        tma_load_3d(sQPe, &tmQ, &bar->qpe_full, kC, 0, row);
+        qpe_armed = ++pc;
         it.next();
-      }
-      if (armed && guard.aborted()) {
-        int dummy = 0;
-        Guard drain{reinterpret_cast<volatile int*>(&dummy), p.status};
-        mbar_wait(&bar->qpe_full, (pc - 1) & 1, drain);
       }
     }
   } else if (warp == 1) {
@@ -438,25 +407,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = true;
       while (ok && it.get(row, k0, k1, nrow, first_row)) {
         const int ntiles = (k1 - k0 + kNK - 1) / kNK;
-        // the piece's latent query → TMEM, once the previous piece's score MMAs have read the old
-        // one (its rotary columns are reloaded by the producer after the same point)
+        // the piece's latent query half → TMEM, once the previous piece's score MMAs have read the
+        // old one (its rotary slab is reloaded by the producer after the same point)
         if (pc > 0 && !mbar_wait(&bar->q_empty, (pc - 1) & 1, guard)) break;
-        for (int qs = 0; qs < kQStages && ok; ++qs, ++rs) {
+        for (int i = 0; i < 4 && ok; ++i, ++rs) {
           const int s = rs % kStages;
           if (!mbar_wait(&bar->kv_full[s], (rs / kStages) & 1, guard)) { ok = false; break; }
           tc_fence_after();
-          for (int h = 0; h < 2; ++h) {
-            const int i = 2 * qs + h;   // latent query slab (64 columns)
-            const uint32_t q0 = smem_u32(sKV + s * kStageBytes + h * kSlabQ);
+          const uint32_t q0 = smem_u32(sKV + s * kStageBytes);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              tmem_cp_128x256b(tmem + kTmemQ + i * 32 + kk * 8,
-                               smem_desc_sw128(q0 + kk * 32, 16, 1024));
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            tmem_cp_128x256b(tmem + kTmemQ + i * 32 + kk * 8, smem_desc_sw128(q0 + kk * 32, 16, 1024));
           umma_commit(&bar->kv_empty[s]);
         }
         if (!ok) break;
-        if (!mbar_wait(&bar->qpe_full, pc & 1, guard)) break;
+        if (rank == 1 && !mbar_wait(&bar->qpe_full, pc & 1, guard)) break;
         const int rs0 = rs;
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
           const int s = (rs0 + j) % kStages, sb = g % kNS;
@@ -467,22 +432,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          // scores: S[128 x 64] = Q_part x K_part^T over this CTA's 288 columns: the latent part
-          // with the query in TMEM, the rotary part with the query in shared memory
+          // scores: S[128 x 32] = Q_half x K_half^T: latent part with the query in TMEM, the
+          // rotary part (rank 1) with the query slab in shared memory; cache K-major in smem
           const uint32_t kv0 = smem_u32(sKV + s * kStageBytes);
-          const uint32_t d = tmem + kTmemS + sb * kNK;
           for (int i = 0; i < 4; ++i) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              umma_bf16_tmem_a(d, tmem + kTmemQ + i * 32 + kk * 8,
+              umma_bf16_tmem_a(tmem + kTmemS + sb * kNK, tmem + kTmemQ + i * 32 + kk * 8,
                                smem_desc_sw128(kv0 + i * kSlabKV + kk * 32, 16, 1024), idesc_qk,
                                (i | kk) != 0);
             }
           }
+          if (rank == 1) {
 #pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            umma_bf16(d, smem_desc_sw64(qpe0 + kk * 32, 512),
-                      smem_desc_sw64(kv0 + 4 * kSlabKV + kk * 32, 512), idesc_qk, 1u);
+            for (int kk = 0; kk < 4; ++kk) {
+              umma_bf16(tmem + kTmemS + sb * kNK, smem_desc_sw128(qpe0 + kk * 32, 16, 1024),
+                        smem_desc_sw128(kv0 + 4 * kSlabKV + kk * 32, 16, 1024), idesc_qk, 1u);
+            }
           }
           umma_commit(&bar->s_full[g % kNB]);
           if (j == ntiles - 1) umma_commit(&bar->q_empty);
@@ -507,7 +473,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = true;
       while (ok && it.get(row, k0, k1, nrow, first_row)) {
         const int ntiles = (k1 - k0 + kNK - 1) / kNK;
-        const int rs0 = g + kQStages * (pc + 1);   // ring slot of the piece's first tile
+        const int rs0 = g + 4 * (pc + 1);   // ring slot of the piece's first tile
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
           const int sb = g % kNS, s = (rs0 + j) % kStages;
           if (!mbar_wait(&bar->p_full[sb], (g / kNS) & 1, guard)) { ok = false; break; }
@@ -535,12 +501,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- softmax, epilogue
     // kGroups groups of four warps take turns by tile (group = global tile index % kGroups);
-    // within a group a thread owns one head row (TMEM lane) and all 64 keys of its tiles.  The
+    // within a group a thread owns one head row (TMEM lane) and all 32 keys of its tiles.  The
     // running maximum of a row is handed from tile to tile across the groups through m_ref / seq
     // in shared memory; each group keeps its own partial row sum relative to the last maximum it
     // used, so the groups' softmax work overlaps and only the max decision is sequential.
+    //
+    // Staging: the four warps of a lane quarter (one per group) share one 4 KB slot for their
+    // outgoing score copies and for the epilogue's TMA stores.  Uses of a slot are numbered in a
+    // fixed order (the pieces' tiles, then each piece's epilogue blocks, group 0 before group 1)
+    // and handed on through a release counter: use u waits until u uses have released it.
     const int quad = warp & 3;
-    const int grp = (warp - kSoftmaxWarp0) >> 2;             // warps 3-6, 7-10
+    const int grp = (warp - kSoftmaxWarp0) >> 2;             // warps 3-6, 7-10, 11-14
     const int lane = static_cast<int>(lane_id());
     const int h = quad * 32 + lane;                          // head row = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
@@ -549,16 +520,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     volatile float* m_ref = reinterpret_cast<volatile float*>(sRed);            // [128]
     volatile int* seq = reinterpret_cast<volatile int*>(sRed + 128);            // [128]
     float* lsum_x = sRed + 256;                       // [piece parity][kGroups][128]
-    const int xw = grp * 4 + quad;                    // this warp's receive slot / barriers
+    uint8_t* stg = sY + quad * kXWarp;                       // this lane quarter's staging slot
+    const int xw = grp * 4 + quad;                           // this warp's receive slot / barriers
     uint8_t* xslot = sX + xw * kXWarp;
     const uint32_t x_remote = mapa_shared(smem_u32(xslot), peer);
     const uint32_t xfull_remote = mapa_shared(smem_u32(&bar->x_full[xw]), peer);
     const uint32_t xempty_remote = mapa_shared(smem_u32(&bar->x_empty[xw]), peer);
-    // row r of a warp's 8 KB score block: 64 floats = 16 chunks of 16 B, chunk c at c ^ (r & 7)
-    auto xoff = [](int r, int c) -> uint32_t {
-      return static_cast<uint32_t>(r * 256 + ((c ^ (r & 7)) << 4));
+    // row r of a warp's 4 KB score block: 32 floats = 8 chunks of 16 B, chunk c at (c + r) & 7
+    auto xoff = [](int r, int c) -> int { return r * 128 + (((c + r) & 7) << 4); };
+    volatile int* y_released = bar->y_released + quad;
+    auto acquire_stage = [&](int u) -> bool {   // wait until uses 0..u-1 released the slot
+      bool got = true;
+      if (*y_released < u) {
+        const unsigned long long t0 = globaltimer_ns();
+        uint32_t n = 0;
+        while (*y_released < u) {
+          if ((++n & 63u) == 0 && (guard.aborted() || globaltimer_ns() - t0 > guard.limit_ns)) {
+            if (!guard.aborted()) guard.fail(kDevTimeout);
+            got = false;
+            break;
+          }
+        }
+      }
+      got = __all_sync(0xffffffffu, got);
+      __threadfence_block();
+      return got;
     };
-    int g = 0, pc = 0;   // tiles before this piece, pieces
+    auto release_stage = [&](int u) {           // the slot's copy / store has read it: hand on
+      if (lane == 0) {
+        bulk_wait_read_all();
+        __threadfence_block();
+        *y_released = u + 1;
+      }
+    };
+    int g = 0, pc = 0, ubase = 0;   // tiles before this piece, pieces, extra slot uses before
     int row, k0, k1, nrow;
     bool first_row;
     bool ok = true;
@@ -575,29 +570,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int ntiles = (k1 - k0 + kNK - 1) / kNK;
       const int g0 = g;
       // ring slot of the piece's first tile: every piece so far (this one included) put its
-      // query stages into the ring ahead of its tiles
-      const int rs0 = g0 + kQStages * (pc + 1);
+      // four query slabs into the ring ahead of its tiles
+      const int rs0 = g0 + 4 * (pc + 1);
       const bool whole = (k0 == 0 && k1 == nrow);
+      constexpr int nblk = 2;           // epilogue blocks of 64 columns per writing group
+      // group 1 stages its epilogue in its own receive slot when it had a tile in this piece (the
+      // peer may refill that slot only after the epilogue: its last release is held back);
+      // otherwise it queues on the lane quarter's shared slot behind group 0
+      const bool g1_has_tile = ((1 - g0 % kGroups + kGroups) % kGroups) < ntiles;
+      bool xe_held = false;
 
       float l_g = 0.f;              // this group's partial row sum ...
       float m_used = -INFINITY;     // ... relative to this maximum
       int j = ((grp - g0 % kGroups) + kGroups) % kGroups;
       for (; j < ntiles; j += kGroups) {
         const int t = g0 + j;
-        const int k = t / kGroups;  // this warp's exchange count (receive-slot phases)
+        const int k = t / kGroups;  // per-group tile counter (exchange slot phases)
         // scores of this CTA's columns
         if (!warp_wait(&bar->s_full[t % kNB], (t / kNB) & 1, guard)) { ok = false; break; }
         tc_fence_after();
         float s[kNK];
-        tmem_ld64(tmem + lane_off + kTmemS + (t % kNS) * kNK, s);
-        // hand this row's 64 partial scores to the peer (its receive slot for this warp), once
-        // the peer has consumed the previous ones
-        if (k >= 1 && !warp_wait<true>(&bar->x_empty[xw], (k - 1) & 1, guard)) { ok = false; break; }
+        tmem_ld32(tmem + lane_off + kTmemS + (t % kNS) * kNK, s);
+        // hand this warp's 32 rows to the peer: stage locally, one 4 KB bulk copy per warp
+        if (!acquire_stage(t + ubase)) { ok = false; break; }
 #pragma unroll
         for (int c = 0; c < kNK / 4; ++c)
-          st_async_v4(x_remote + xoff(lane, c), __float_as_uint(s[4 * c]),
-                      __float_as_uint(s[4 * c + 1]), __float_as_uint(s[4 * c + 2]),
-                      __float_as_uint(s[4 * c + 3]), xfull_remote);
+          *reinterpret_cast<float4*>(stg + xoff(lane, c)) =
+              make_float4(s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (k >= 1 && !mbar_wait<true>(&bar->x_empty[xw], (k - 1) & 1, guard)) ok = false;
+          if (ok) {
+            bulk_copy_to_peer(x_remote, smem_u32(stg), kXWarp, xfull_remote);
+            bulk_commit();
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        release_stage(t + ubase);   // as soon as the copy has read the slot
         // the peer's half of the same tile
         if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[xw], kXWarp);
         if (!warp_wait<true>(&bar->x_full[xw], k & 1, guard)) { ok = false; break; }
@@ -610,37 +621,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           s[4 * c + 3] += x.w;
         }
         // every lane has consumed its loads from the slot before lane 0 lets the peer refill it
-        consume32(*reinterpret_cast<const float(*)[32]>(&s[0]));
-        consume32(*reinterpret_cast<const float(*)[32]>(&s[32]));
+        consume32(s);
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote_relaxed(xempty_remote);
+        if (grp == 1 && j + kGroups >= ntiles) xe_held = true;   // released after the epilogue
+        else if (lane == 0) mbar_arrive_remote_relaxed(xempty_remote);
         const int key0 = k0 + j * kNK;
         const int nvalid = min(kNK, k1 - key0);
-        if (p.logits && rank == 0 && h < p.n_heads) {
+        if (p.logits && rank == 0 && h < p.n_heads && key0 >= 0 && !p.topk_idx) {
           float* lg =
               p.logits + (static_cast<size_t>(row) * p.n_heads + h) * p.max_seq_len + key0;
 #pragma unroll
           for (int i = 0; i < kNK; ++i)
-            if (i < nvalid) lg[i] = s[i] * p.scale;
+            if (i < nvalid && key0 + i < p.max_seq_len) lg[i] = s[i] * p.scale;
         }
         // the tile maximum on unscaled scores (the scale is positive: it commutes with max); the
         // exp2 below applies the scale in its FMA
+        float mx[8];
         const float c2 = p.scale_log2;
 #pragma unroll
         for (int i = 0; i < kNK; ++i) s[i] = i < nvalid ? s[i] : -INFINITY;
-        float mx[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          mx[i] = fmaxf(fmaxf(s[i], s[i + 16]), fmaxf(s[i + 32], s[i + 48]));
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], mx[i + 8]);
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(fmaxf(s[i], s[i + 8]), fmaxf(s[i + 16], s[i + 24]));
 #pragma unroll
         for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
         const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c2;
-        // running-max decision for tile t (after the other group decided tile t-1)
+        // running-max decision for tile t (after another group decided tile t-1)
         float m_prev = -INFINITY;
         if (j > 0) {
-          if (!wait_seq(seq, h, t - 1, guard)) { ok = false; break; }
+          bool seen = true;
+          if (seq[h] != t - 1) {
+            const unsigned long long t0 = globaltimer_ns();
+            uint32_t n = 0;
+            while (seq[h] != t - 1) {
+              if ((++n & 63u) == 0 &&
+                  (guard.aborted() || globaltimer_ns() - t0 > guard.limit_ns)) {
+                if (!guard.aborted()) guard.fail(kDevTimeout);
+                seen = false;
+                break;
+              }
+            }
+          }
+          if (!__all_sync(0xffffffffu, seen)) { ok = false; break; }
           __threadfence_block();
           m_prev = m_ref[h];
         }
@@ -682,19 +703,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < kNK / 2; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] += s[i + 32];
-#pragma unroll
         for (int i = 0; i < 16; ++i) s[i] += s[i + 16];
 #pragma unroll
         for (int i = 0; i < 8; ++i) s[i] += s[i + 8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) s[i] += s[i + 4];
         l_g += (s[0] + s[2]) + (s[1] + s[3]);
-        tmem_st32_u32(tmem + lane_off + kTmemS + (t % kNS) * kNK, pk);
+        tmem_st16_u32(tmem + lane_off + kTmemS + (t % kNS) * kNK, pk);
         if (nvalid < kNK) {
           // keys past the piece's end: zero their latent rows so garbage cannot reach P·V
           uint8_t* st = sKV + ((rs0 + j) % kStages) * kStageBytes;
-          const int per_slab = (kNK - nvalid) * 8;   // 16-byte chunks per slab
+          const int per_slab = (kNK - nvalid) * 8;
           for (int q = gtid; q < per_slab * 4; q += 128) {
             const int slab = q / per_slab;
             const int rem = q - slab * per_slab;
@@ -712,7 +731,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------ epilogue of the piece
       const int glast = g - 1;
       // final maximum of the row (decided at the last tile), all groups' sums relative to it
-      if (!wait_seq(seq, h, glast, guard)) break;
+      {
+        bool seen = true;
+        const unsigned long long t0 = globaltimer_ns();
+        uint32_t n = 0;
+        while (seq[h] != glast) {
+          if ((++n & 63u) == 0 && (guard.aborted() || globaltimer_ns() - t0 > guard.limit_ns)) {
+            if (!guard.aborted()) guard.fail(kDevTimeout);
+            seen = false;
+            break;
+          }
+        }
+        if (!__all_sync(0xffffffffu, seen)) break;
+      }
       __threadfence_block();
       const float m_fin = m_ref[h];
       // (double-buffered by piece: a group cannot pass the next piece's sync_all before every
@@ -726,44 +757,78 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float inv_l = 1.f / l_tot;
       const float lse = (m_fin + log2f(l_tot)) * 0.69314718055994531f;
       const int slot = first_row ? 0 : 1;
-      // group G writes columns [128G, 128G + 128) of the CTA's 256: bf16 o_lat for an uncut row,
-      // fp16 normalised partials for a cut one, 64 bytes per thread and block, from registers
-      if (!warp_wait(&bar->pv_done[glast % kNB], (glast / kNB) & 1, guard)) break;
-      tc_fence_after();
-      const int ocol = col0 + grp * 128;
-      const bool write_row = whole ? (h < p.n_heads) : true;
-      uint4* dst = whole
-                       ? reinterpret_cast<uint4*>(p.o_lat +
-                                                  (static_cast<size_t>(row) * p.n_heads + h) * kC + ocol)
-                       : reinterpret_cast<uint4*>(p.part_o +
-                                                  ((static_cast<size_t>(pair) * 2 + slot) * 128 + h) * kC + ocol);
+      if (grp < 2) {
+        // Groups 0 and 1 write the CTA's 256 columns of O (128 each) in blocks of 32 rows x 64
+        // columns (bf16 for an uncut row, fp16 normalised partials for a cut one: 128-byte rows),
+        // staged in the 128-byte-swizzle layout (lane = row, chunk c at c ^ (row & 7)), one TMA
+        // tile store per block; the warps do not wait for the global writes.
+        if (!warp_wait(&bar->pv_done[glast % kNB], (glast / kNB) & 1, guard)) break;
+        tc_fence_after();
+        const int ocol = col0 + grp * 128;
+        const bool own_slot = (grp == 1 && xe_held);
+        uint8_t* est = own_slot ? xslot : stg;
+        const int u0 = g + ubase + grp * nblk;   // shared-slot uses (group 1: only if queued)
 #pragma unroll 1
-      for (int blk = 0; blk < 4; ++blk) {
-        float v[32];
-        tmem_ld32(tmem + lane_off + kTmemO + grp * 128 + blk * 32, v);
-        uint32_t w[16];
+        for (int blk = 0; blk < nblk; ++blk) {
+          uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = whole ? pack_bf16x2(v[2 * i] * inv_l, v[2 * i + 1] * inv_l)
-                       : pack_f16x2(v[2 * i] * inv_l, v[2 * i + 1] * inv_l);
-        if (write_row) {
+          for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tmem_ld32(tmem + lane_off + kTmemO + grp * 128 + blk * 64 + half * 32, v);
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            dst[blk * 4 + c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+            for (int i = 0; i < 16; ++i)
+              w[16 * half + i] = whole ? pack_bf16x2(v[2 * i] * inv_l, v[2 * i + 1] * inv_l)
+                                       : pack_f16x2(v[2 * i] * inv_l, v[2 * i + 1] * inv_l);
+          }
+          if (blk == nblk - 1) {   // every TMEM read of O is done: the next piece may overwrite it
+            tc_fence_before();
+            mbar_arrive(&bar->o_empty);
+          }
+          if (own_slot) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+          } else if (!acquire_stage(u0 + blk)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(est + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (whole) {
+              if (quad * 32 < p.n_heads) tma_store_3d(&tmO, est, ocol + blk * 64, quad * 32, row);
+            } else {
+              tma_store_2d(&tmPart, est, ocol + blk * 64, (pair * 2 + slot) * 128 + quad * 32);
+            }
+            bulk_commit();
+          }
+          if (!own_slot) release_stage(u0 + blk);
         }
+        if (!ok) break;
+        if (own_slot) {   // the stores have read the slot: the peer may refill it
+          if (lane == 0) {
+            bulk_wait_read_all();
+            mbar_arrive_remote_relaxed(xempty_remote);
+          }
+          xe_held = false;
+        }
+      } else {
+        mbar_arrive(&bar->o_empty);   // this group reads no O
       }
-      // every TMEM read of O is done: the next piece may overwrite it
-      tc_fence_before();
-      mbar_arrive(&bar->o_empty);
       if (whole) {
         if (rank == 0 && grp == 0 && p.lse_out && h < p.n_heads)
           p.lse_out[static_cast<size_t>(row) * p.n_heads + h] = lse;
       } else if (rank == 0 && grp == 0) {
         p.part_lse[(static_cast<size_t>(pair) * 2 + slot) * 128 + h] = lse;
       }
+      ubase += g1_has_tile ? nblk : 2 * nblk;
       ++pc;
       it.next();
     }
+    if (lane == 0) bulk_wait_all();   // every copy and store this warp issued has completed
   }
 
   // ------------------------------------------------------------------ teardown
@@ -774,6 +839,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (guard.aborted()) {   // every role has stopped: let the loads this thread armed land
+    int dummy = 0;
+    Guard drain{reinterpret_cast<volatile int*>(&dummy), p.status};
+    for (int s = 0; s < kStages; ++s)
+      if (last_slot[s] >= 0) mbar_wait(&bar->kv_full[s], (last_slot[s] / kStages) & 1, drain);
+    if (qpe_armed > 0) mbar_wait(&bar->qpe_full, (qpe_armed - 1) & 1, drain);
+  }
   cluster_sync_all();   // no remote access into this CTA's shared memory is still pending
   if (warp == 1) {
     tc_fence_after();
@@ -798,7 +870,7 @@ cudaError_t attention_prepare() {
 cudaError_t launch_attention(const AttnMaps& m, const AttnParams& p, int n_pairs, cudaStream_t s,
                              bool pdl) {
   LaunchCfg lc(dim3(2 * n_pairs), dim3(kThreads), kAttnSmem, s, pdl);
-  return cudaLaunchKernelEx(&lc.cfg, latent_attention_kernel, m.kv, m.pe, m.q, m.qpe,
+  return cudaLaunchKernelEx(&lc.cfg, latent_attention_kernel, m.kv, m.pe, m.q, m.o, m.part,
                             p.topk_idx ? m.kv2 : m.kv, p.topk_idx ? m.pe2 : m.pe, p);
 }
 
@@ -809,32 +881,36 @@ bool make_gather_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st,
   if (rows >= (1ull << 31)) return false;   // gather row coordinates are 32-bit
   const uint64_t d_kv[2] = {kC, rows}, s_kv[1] = {static_cast<uint64_t>(kv_st) * 2};
   const uint64_t d_pe[2] = {kDr, rows}, s_pe[1] = {static_cast<uint64_t>(pe_st) * 2};
-  const uint32_t box_kv[2] = {64, 1}, box_pe[2] = {32, 1};
-  return encode_tiled(&m->kv2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv, d_kv, s_kv, box_kv,
+  const uint32_t box[2] = {64, 1};
+  return encode_tiled(&m->kv2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv, d_kv, s_kv, box,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
-         encode_tiled(&m->pe2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pe, d_pe, s_pe, box_pe,
-                      CU_TENSOR_MAP_SWIZZLE_64B);
+         encode_tiled(&m->pe2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pe, d_pe, s_pe, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,
                          int64_t pe_sb, int64_t pe_st, int batch, int max_seq_len, const void* qabs,
-                         int rows) {
+                         int rows, const void* o_lat, int n_heads, const void* part_o, int pairs) {
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
   const uint64_t L = static_cast<uint64_t>(max_seq_len), Bt = static_cast<uint64_t>(batch);
-  const uint64_t R = static_cast<uint64_t>(rows);
+  const uint64_t R = static_cast<uint64_t>(rows), H = static_cast<uint64_t>(n_heads);
   const uint32_t box_kv[3] = {64, static_cast<uint32_t>(kNK), 1};
-  const uint32_t box_pe[3] = {32, static_cast<uint32_t>(kNK), 1};
   const uint64_t d_kv[3] = {kC, L, Bt}, s_kv[2] = {static_cast<uint64_t>(kv_st) * 2,
                                                    static_cast<uint64_t>(kv_sb) * 2};
   const uint64_t d_pe[3] = {kDr, L, Bt}, s_pe[2] = {static_cast<uint64_t>(pe_st) * 2,
                                                     static_cast<uint64_t>(pe_sb) * 2};
   const uint64_t d_q[3] = {kDk, kHPad, R}, s_q[2] = {kDk * 2, kHPad * kDk * 2};
   const uint32_t box_q[3] = {64, 128, 1};
-  const uint32_t box_qpe[3] = {32, 128, 1};
-  return encode_tiled(&m->kv, bf, 3, kv, d_kv, s_kv, box_kv, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         encode_tiled(&m->pe, bf, 3, pe, d_pe, s_pe, box_pe, CU_TENSOR_MAP_SWIZZLE_64B) &&
-         encode_tiled(&m->q, bf, 3, qabs, d_q, s_q, box_q, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         encode_tiled(&m->qpe, bf, 3, qabs, d_q, s_q, box_qpe, CU_TENSOR_MAP_SWIZZLE_64B);
+  const uint64_t d_o[3] = {kC, H, R}, s_o[2] = {kC * 2, H * kC * 2};
+  const uint32_t box_o[3] = {64, 32, 1};
+  const uint64_t d_p[2] = {kC, static_cast<uint64_t>(pairs) * 2 * 128}, s_p[1] = {kC * 2};
+  const uint32_t box_p[2] = {64, 32};
+  return encode_tiled(&m->kv, bf, 3, kv, d_kv, s_kv, box_kv, sw) &&
+         encode_tiled(&m->pe, bf, 3, pe, d_pe, s_pe, box_kv, sw) &&
+         encode_tiled(&m->q, bf, 3, qabs, d_q, s_q, box_q, sw) &&
+         encode_tiled(&m->o, bf, 3, o_lat, d_o, s_o, box_o, sw) &&
+         encode_tiled(&m->part, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, part_o, d_p, s_p, box_p, sw);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -853,10 +929,14 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineP
   for (int task = blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5);
        task < p.rows * p.n_heads; task += warps) {
   const int r = task / p.n_heads, h = task - r * p.n_heads;
-  const int2 pcs = p.row_pieces[r];
+  const int2 pcs = __ldcg(p.row_pieces + r);
   const int plo = pcs.x >> 1, phi = pcs.y;
   const int slot_lo = pcs.x & 1;   // the first piece is the tail of a pair begun in an earlier row
   if (plo == phi) continue;   // written by one pair
+  if (plo < 0 || phi < plo || phi >= p.n_pairs) {   // not a record the key prefix can produce
+    if (lane == 0) atomicCAS(p.status, kDevOk, kDevBadArg);
+    continue;
+  }
   // online log-sum-exp merge, four pieces' loads in flight at a time
   constexpr int kBatch = 4;
   float mx = -INFINITY, wsum = 0.f;

@@ -98,7 +98,13 @@ __device__ void build_merged_b(const GemmParams& p, int g, int n0, uint8_t* sBm,
 #pragma unroll
   for (int k = 0; k < kPre; ++k) {
     const int n = n0 + lane + 32 * k;
-    pre[k] = n < p.N ? p.row_pieces[n] : make_int2(0, 0);
+    pre[k] = n < p.N ? __ldcg(p.row_pieces + n) : make_int2(0, 0);
+    // a record the key prefix cannot produce is reported and read as "one piece"
+    const int lo = pre[k].x >> 1, hi = pre[k].y;
+    if (n < p.N && (lo < 0 || hi < lo || hi >= p.n_pairs)) {
+      atomicCAS(p.status, kDevOk, kDevBadArg);
+      pre[k] = make_int2(0, 0);
+    }
   }
   auto pieces_of = [&](int i) -> int2 {   // row_pieces[n0 + i], 0 <= i < BN (warp-uniform i)
     int2 v = make_int2(0, 0);
@@ -363,6 +369,7 @@ __global__ void __launch_bounds__(gemm_threads<FP8>(), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  int issued = 0;   // producer thread: ring slots whose loads it issued
 
   if (warp == 0) {
     if (elect_one()) {
@@ -404,13 +411,7 @@ __global__ void __launch_bounds__(gemm_threads<FP8>(), 1)
                         un.n0);
         }
       }
-      if (guard.aborted()) {
-        // drain the loads still in flight before the CTA's shared memory goes away
-        int dummy = 0;
-        Guard dr{reinterpret_cast<volatile int*>(&dummy), p.status};
-        for (int k = ks > STAGES ? ks - STAGES : 0; k < ks; ++k)
-          mbar_wait(&full[k % STAGES], (k / STAGES) & 1, dr);
-      }
+      issued = ks;   // slots [0, ks) were armed and loaded (a failed slot breaks before)
     }
   } else if (warp == 1) {
     if (elect_one()) {
@@ -453,10 +454,16 @@ __global__ void __launch_bounds__(gemm_threads<FP8>(), 1)
     bool ok = true;
     while (ok && sched.next(u)) {
       const Unit un = unit_of(u, mt, nt, BN);
-      const float* sc = p.a_scale + un.g * p.a_sg + ((un.m0 + p.a_row_off) >> 7) * p.a_sm;
+      const long long sc0 = un.g * p.a_sg + ((un.m0 + p.a_row_off) >> 7) * p.a_sm;
       for (int j = 0; j < nk; ++j, ++ks) {
         const int s = ks % STAGES;
-        const float scale = __ldg(sc + ((j * 64) >> 7) * p.a_sk);
+        const long long si = sc0 + ((j * 64) >> 7) * p.a_sk;
+        float scale = 0.f;
+        if (si >= 0 && si < p.a_scale_n) {
+          scale = __ldg(p.a_scale + si);
+        } else if (ctid == 0) {
+          guard.fail(kDevBadArg);   // a scale index outside the tensor: reported, not read
+        }
         if (!mbar_wait(&full[s], (ks / STAGES) & 1, guard)) { ok = false; break; }
         const uint8_t* src = sA8 + s * kSlabA8;
         uint8_t* dst = sA + s * kSlabA;
@@ -540,6 +547,14 @@ __global__ void __launch_bounds__(gemm_threads<FP8>(), 1)
 
   tc_fence_before();
   __syncthreads();
+  if (issued > 0 && guard.aborted()) {
+    // a role gave up (possibly after the producer had issued everything): the ring's last loads
+    // may still be in flight, so they land before the CTA's shared memory goes away
+    int dummy = 0;
+    Guard dr{reinterpret_cast<volatile int*>(&dummy), p.status};
+    for (int k = issued > STAGES ? issued - STAGES : 0; k < issued; ++k)
+      mbar_wait(&full[k % STAGES], (k / STAGES) & 1, dr);
+  }
   if (warp == 1) {
     int dummy = 0;
     Guard dr{reinterpret_cast<volatile int*>(&dummy), p.status};

@@ -96,7 +96,7 @@ extern "C" mla_status mla_latent_attention_noalloc(
   const int pairs = attention_pairs() < kNoAllocPairs ? attention_pairs() : kNoAllocPairs;
   AttnMaps am;
   if (!make_attention_maps(&am, kv_cache, kv_stride_b, kv_stride_t, pe_cache, pe_stride_b,
-                           pe_stride_t, rows, max_seq_len, q_abs, rows))
+                           pe_stride_t, rows, max_seq_len, q_abs, rows, o_lat, n_heads, part_o, pairs))
     return MLA_ERR_INVALID_ARG;
 
   // the prefix and partials in the scratch array are written before they are read within the
@@ -143,6 +143,7 @@ extern "C" mla_status mla_latent_attention_noalloc(
   cp.row_pieces = row_pieces;
   cp.o_lat = static_cast<bf16*>(o_lat);
   cp.lse_out = lse;
+  cp.status = st;
   if (launch_combine(cp, stream, false) != cudaSuccess) return MLA_ERR_CUDA;
   return MLA_OK;
 }

@@ -120,7 +120,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   const uint32_t a = smem_u32(bar);
   if (kClusterAcquire ? mbar_test_cluster(a, parity) : mbar_test(a, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
-  uint32_t n = 0;
+  uint32_t n = 63;   // the first failed poll already checks the clock (short limits apply)
   while (true) {
     if (kClusterAcquire ? mbar_test_cluster(a, parity) : mbar_test(a, parity)) return true;
     if ((++n & 63u) == 0) {
