@@ -288,6 +288,9 @@ def run_workload(name: str, args, rank: int, world: int, local_rank: int,
     del inp
     rt = MLARuntime(gamma, wq_b, wkv_b, n_heads=H, max_rows=B * T, max_seq_len=cache.shape[1],
                     rope_theta=w.rope_theta, rms_eps=w.rms_eps, **scales)
+    # the set-up kernels (workspace zeroing, W_UK^T copy) ran on the current stream; the timed
+    # calls use a pool stream that does not wait for it
+    torch.cuda.synchronize()
     out_shape = (B, H, 128) if w.mode == "decode" else (B, T, H, 128)
     out = torch.empty(out_shape, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -510,6 +513,7 @@ def run_producer(name: str, args, rank: int, world: int, local_rank: int) -> dic
     rt = MLARuntime(gamma, wq_b, wkv_b, n_heads=w.dims.n_heads, max_rows=B * T,
                     max_seq_len=cache.shape[1], rope_theta=w.rope_theta, rms_eps=w.rms_eps)
     rt.attach_producer(wq_a, wkv_a, kv_gain)
+    torch.cuda.synchronize()   # set-up kernels ran on the current stream (see run_workload)
     q_lat = torch.empty(B, T, 1536, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -782,11 +786,18 @@ def main(argv=None):
     names = WORKLOAD_ORDER if args.workload == "all" else (args.workload,)
     entries = {n: run_workload(n, args, rank, world, local_rank) for n in names}
     if args.workload == "all":
+        # the variants and the producer are measured beside the configurations; a failure in one
+        # of them is reported in its entry instead of voiding the line
+        def guarded(fn, *a, **kw):
+            try:
+                return fn(*a, **kw)
+            except Exception as e:  # noqa: BLE001
+                return {"error": f"{type(e).__name__}: {e}"[:300], "gpu_launches": 0}
         for n, (base, variant) in VARIANTS.items():
-            entries[n] = run_workload(base, args, rank, world, local_rank, variant=variant,
-                                      entry=n)
+            entries[n] = guarded(run_workload, base, args, rank, world, local_rank,
+                                 variant=variant, entry=n)
         for n in PRODUCER_RUNS:
-            entries[n] = run_producer(n, args, rank, world, local_rank)
+            entries[n] = guarded(run_producer, n, args, rank, world, local_rank)
     if rank == 0:
         head_name = names[0]
         head = entries[head_name]
@@ -810,7 +821,8 @@ def main(argv=None):
                                      "every workload below (headline included)")
         if not args.no_cpu_baseline and world == 1 and args.workload == "all":
             for n in PRODUCER_RUNS:
-                entries[n]["cpu_baseline"] = producer_oracle_sample(n, min(4.0, args.cpu_seconds))
+                if entries[n] and "error" not in entries[n]:
+                    entries[n]["cpu_baseline"] = producer_oracle_sample(n, min(4.0, args.cpu_seconds))
         if len(names) > 1:
             line["workloads"] = {n: entries[n] for n in entries if n != head_name}
         print(json.dumps(line), flush=True)
