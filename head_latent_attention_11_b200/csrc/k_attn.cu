@@ -315,7 +315,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // rotary query slab into its own buffer, once the previous piece's last score MMA has read it.
     const uint32_t lane = lane_id();
     if (lane == 0 && !p.topk_idx) {
-      const uint64_t pol = policy_evict_first();
+      // decode reads each cache row once (evict first); a prefill chunk's rows all re-read the
+      // same key prefix, which should stay in L2 (evict last, and no look-ahead: after the first
+      // row's pass every tile is an L2 hit)
+      const bool reread = p.T > 1;
+      const uint64_t pol = reread ? policy_evict_last() : policy_evict_first();
       // L2 look-ahead: a second cursor over the same tiles, kL2Ahead tiles in front of the ring
       // loads, has the TMA unit pull its tiles into L2, so the bytes in flight from HBM are not
       // limited by the ring's depth.  Its first kL2Ahead tiles go out before the wait below.
@@ -324,7 +328,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ring can be filled; the tiles in between load from HBM within the ring's depth (every
       // tile: 0.83 us per tile; every other: 68.5 us per launch; one in three: 67.0 us).
       PieceIter pf = it;
-      bool pf_live = false, pf_done = false;
+      bool pf_live = false, pf_done = reread;
       int pf_b = 0, pf_key = 0, pf_end = 0, pf_n = 0;
       auto prefetch_next = [&]() {
         while (!pf_done) {
