@@ -34,12 +34,15 @@ namespace {
 
 constexpr int kEpiWarps = 8;                            // two per TMEM lane quadrant
 constexpr int kEpiThreads = 32 * kEpiWarps;
-constexpr int kConvThreads = 128;                       // FP8: four converter warps
+// FP8: converter threads — four warps; two in the merge mode, whose B builder needs the registers
+// (a block of more than 384 threads is held to 128 registers a thread)
+template <bool MERGE>
+__host__ __device__ constexpr int conv_threads() { return MERGE ? 64 : 128; }
 constexpr int kSlabA = 128 * 64 * 2;   // 16 KB
 constexpr int kSlabA8 = 128 * 64;      // 8 KB: an FP8 weight slab (64-byte rows, no swizzle)
 
-template <bool FP8>
-constexpr int gemm_threads() { return 64 + kEpiThreads + (FP8 ? kConvThreads : 0); }
+template <bool FP8, bool MERGE = false>
+constexpr int gemm_threads() { return 64 + kEpiThreads + (FP8 ? conv_threads<MERGE>() : 0); }
 
 template <int BN>
 struct GemmTile {
@@ -311,7 +314,7 @@ struct Sched {
 };
 
 template <int BN, int STAGES, bool MERGE, bool FP8>
-__global__ void __launch_bounds__(gemm_threads<FP8>(), 1)
+__global__ void __launch_bounds__(gemm_threads<FP8, MERGE>(), 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmParams p, const int batches) {
   extern __shared__ uint8_t smem_raw[];
@@ -358,7 +361,7 @@ __global__ void __launch_bounds__(gemm_threads<FP8>(), 1)
     mbar_init(drain, 1);
     mbar_init(b_ready, kEpiThreads);
     if (FP8)
-      for (int i = 0; i < STAGES; ++i) mbar_init(&conv[i], kConvThreads);
+      for (int i = 0; i < STAGES; ++i) mbar_init(&conv[i], conv_threads<MERGE>());
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -446,30 +449,43 @@ __global__ void __launch_bounds__(gemm_threads<FP8>(), 1)
     }
   } else if (FP8 && warp >= 2 + kEpiWarps) {
     // FP8 converter warps: each ring slab of fp8 weight codes → bf16 (code × the block's scale)
-    // in the 128-byte-swizzled layout the MMA reads; thread t converts 16-byte chunks t, t+128,
-    // t+256, t+384 of the slab (row = chunk / 4, 16 columns each)
+    // in the 128-byte-swizzled layout the MMA reads; thread t converts 16-byte chunks t, t + T,
+    // t + 2T, ... of the slab (T converter threads; row = chunk / 4, 16 columns each).  A slab (128 rows x 64
+    // columns) lies in one 128 x 128 scale block.  Lane b of every converter warp holds the scale
+    // of K block b of the current tile and has the next tile's in flight, so no slab waits on a
+    // scale load (the launcher limits FP8 GEMMs to K <= 32 * 128).
     const int ctid = static_cast<int>(threadIdx.x) - (64 + kEpiThreads);
+    const int lane = static_cast<int>(lane_id());
+    const int kblocks = (p.K + 127) / 128;
+    auto tile_scale = [&](int unit) -> float {   // this lane's K block of tile `unit`
+      if (unit < 0 || lane >= kblocks) return 0.f;
+      const Unit un = unit_of(unit, mt, nt, BN);
+      const long long si = un.g * p.a_sg + ((un.m0 + p.a_row_off) >> 7) * p.a_sm + lane * p.a_sk;
+      if (si >= 0 && si < p.a_scale_n) return __ldg(p.a_scale + si);
+      guard.fail(kDevBadArg);   // a scale index outside the tensor: reported, not read
+      return 0.f;
+    };
     int ks = 0;
     int u;
     bool ok = true;
+    Sched ahead = sched;   // one tile ahead of `sched`
+    int u_next = -1;
+    float sc_next = 0.f;
+    if (ahead.next(u_next)) sc_next = tile_scale(u_next);
     while (ok && sched.next(u)) {
-      const Unit un = unit_of(u, mt, nt, BN);
-      const long long sc0 = un.g * p.a_sg + ((un.m0 + p.a_row_off) >> 7) * p.a_sm;
+      const float sc_cur = sc_next;   // tile u's scales (u == u_next)
+      u_next = -1;
+      sc_next = ahead.next(u_next) ? tile_scale(u_next) : 0.f;
       for (int j = 0; j < nk; ++j, ++ks) {
         const int s = ks % STAGES;
-        const long long si = sc0 + ((j * 64) >> 7) * p.a_sk;
-        float scale = 0.f;
-        if (si >= 0 && si < p.a_scale_n) {
-          scale = __ldg(p.a_scale + si);
-        } else if (ctid == 0) {
-          guard.fail(kDevBadArg);   // a scale index outside the tensor: reported, not read
-        }
-        if (!mbar_wait(&full[s], (ks / STAGES) & 1, guard)) { ok = false; break; }
+        const float scale = __shfl_sync(0xffffffffu, sc_cur, (j * 64) >> 7);
+        // voted wait: the warp stays converged for the next shuffle
+        if (!warp_wait(&full[s], (ks / STAGES) & 1, guard)) { ok = false; break; }
         const uint8_t* src = sA8 + s * kSlabA8;
         uint8_t* dst = sA + s * kSlabA;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int ch = ctid + kConvThreads * q;
+        for (int q = 0; q < 512 / conv_threads<MERGE>(); ++q) {   // 512 chunks of 16 bytes
+          const int ch = ctid + conv_threads<MERGE>() * q;
           const int r = ch >> 2, c = ch & 3;
           const uint4 v = *reinterpret_cast<const uint4*>(src + r * 64 + c * 16);
           uint4 lo, hi;
@@ -577,7 +593,7 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Ge
   }
   const int total = batches * ((p.M + 127) / 128) * ((p.N + BN - 1) / BN);
   const int grid = total < g_num_sms ? total : g_num_sms;
-  LaunchCfg lc(dim3(grid), dim3(gemm_threads<FP8>()), gemm_smem_bytes<BN, STAGES, MERGE, FP8>(), s,
+  LaunchCfg lc(dim3(grid), dim3(gemm_threads<FP8, MERGE>()), gemm_smem_bytes<BN, STAGES, MERGE, FP8>(), s,
                pdl);
   return cudaLaunchKernelEx(&lc.cfg, gemm_bf16_kernel<BN, STAGES, MERGE, FP8>, ta, tb, p, batches);
 }
@@ -597,6 +613,7 @@ cudaError_t set_attr() {
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                         int batches, cudaStream_t s, bool pdl) {
   if (p.a_scale) {   // FP8 weights: an 8 KB fp8 slab per stage on top of the bf16 one
+    if (p.K > 32 * 128) return cudaErrorInvalidValue;   // one scale per lane of a warp
     if (p.bmerge) {
       if (p.K != kC || p.N > 64) return cudaErrorInvalidValue;
       if (p.N <= 32) return launch_gemm_t<32, 7, true, true>(ta, tb, p, batches, s, pdl);
