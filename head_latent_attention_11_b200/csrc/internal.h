@@ -212,13 +212,14 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const Gemm
 // Tensor maps of the attention kernel, built on the host for each call (all 128-byte swizzle).
 struct AttnMaps {
   CUtensorMap kv;    // latent cache  bf16 {512, max_seq_len, batch}, box {64, 32, 1}
-  CUtensorMap pe;    // rotary cache  bf16 {64, max_seq_len, batch},  box {64, 32, 1}
+  CUtensorMap pe;    // rotary cache  bf16 {64, max_seq_len, batch},  box {32, 32, 1}, 64-B swizzle
   CUtensorMap q;     // absorbed queries bf16 {576, 128, rows},       box {64, 128, 1}
+  CUtensorMap qpe;   // the same, 64-byte swizzle,                     box {32, 128, 1}
   CUtensorMap o;     // o_lat         bf16 {512, n_heads, rows},      box {64, 32, 1}
   CUtensorMap part;  // split partials fp16 {512, pairs * 2 * 128},   box {64, 32}
   // index-mask decode only: the caches as 2-D row arrays for tile::gather4 (one-row boxes)
   CUtensorMap kv2;   // bf16 {512, batch * seq_rows}, box {64, 1}
-  CUtensorMap pe2;   // bf16 {64, batch * seq_rows},  box {64, 1}
+  CUtensorMap pe2;   // bf16 {64, batch * seq_rows},  box {32, 1}, 64-B swizzle
 };
 // Strides in elements; false if a map cannot be encoded (alignment, sizes).
 bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,

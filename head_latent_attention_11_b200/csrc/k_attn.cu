@@ -10,17 +10,20 @@
 //   * One query row (one token of one sequence) at a time; its heads form the MMA M dimension
 //     (128 rows; heads beyond H are zero rows), so QK^T and P·V are dense 128-row tcgen05 MMAs.
 //   * A cluster of TWO CTAs (one SM each) handles a row.  CTA 0 owns the latent columns
-//     [0, 256); CTA 1 owns [256, 512) and the 64 rotary columns.  Each CTA streams only its
+//     [0, 256) and rotary columns [0, 32); CTA 1 owns [256, 512) and rotary [32, 64), so both
+//     move 18 KB per 32-key tile (with all 64 rotary columns on CTA 1 it moved 20 KB against 16
+//     and set the pace).  Each CTA streams only its
 //     columns of every cache tile (the 576-wide cache row crosses HBM once), computes a partial
 //     score tile over them and hands it to the peer; both CTAs then hold identical full scores
 //     and run the identical online softmax.  Each CTA accumulates the value half it owns,
 //     O[128 x 256] fp32 in TMEM.
-//   * The CTA's 256 latent query columns live in TMEM (A operand of the score MMA); rank 1's 64
+//   * The CTA's 256 latent query columns live in TMEM (A operand of the score MMA); its 32
 //     rotary query columns stay in shared memory (A from a smem descriptor for those K-steps), so
 //     both CTAs have room for four score buffers.  The query reaches TMEM by TMA into ring slots
 //     and tcgen05.cp, once per piece.  The probabilities P (bf16) overwrite the score tile in
-//     TMEM and are the A operand of P·V.  Shared memory holds the cache ring (32-key tiles, 7
-//     stages, TMA with 128-byte swizzle, evict-first) and the exchange buffers.
+//     TMEM and are the A operand of P·V.  Shared memory holds the cache ring (32-key tiles, 8
+//     stages; latent slabs with 128-byte swizzle, rotary half slabs with 64-byte swizzle;
+//     evict-first) and the exchange buffers.
 //     TMEM columns: O [0,256) | latent query [256,384) | four 32-column score/P buffers [384,512).
 //     With four buffers the score MMA of tile g only waits for P·V of tile g-4 to be issued.
 //   * Score exchange: each warp stages its 32 rows of partial scores and ships them with one
@@ -54,7 +57,7 @@ namespace mla {
 namespace {
 
 constexpr int kNK = kAttnKeysPerTile;      // keys per tile
-constexpr int kStages = 7;                 // cache tile ring depth
+constexpr int kStages = 8;                 // cache tile ring depth
 // L2 look-ahead (build-time tuning): tiles it runs ahead of the ring loads, and one tile in
 // kL2Every is prefetched (0: no look-ahead)
 #ifndef MLA_ATTN_L2_AHEAD
@@ -65,18 +68,20 @@ constexpr int kStages = 7;                 // cache tile ring depth
 #endif
 constexpr int kL2Ahead = MLA_ATTN_L2_AHEAD;
 constexpr int kL2Every = MLA_ATTN_L2_EVERY;
-constexpr int kSlabKV = kNK * 128;         // 4 KB: 64 columns x 32 keys, bf16
-constexpr int kMaxSlabs = 5;               // rank 1: 4 latent slabs + 1 rotary slab
+constexpr int kSlabKV = kNK * 128;         // 4 KB: 64 latent columns x 32 keys, bf16
+constexpr int kSlabPe = kNK * 64;          // 2 KB: 32 rotary columns x 32 keys (64-byte rows)
 constexpr int kSlabQ = 128 * 64 * 2;       // 16 KB: 64 query columns of all 128 head rows
-constexpr int kStageBytes = kMaxSlabs * kSlabKV;
+constexpr int kSlabQPe = 128 * 32 * 2;     // 8 KB: this CTA's 32 rotary query columns
+constexpr int kTileBytes = 4 * kSlabKV + kSlabPe;   // 18 KB: a CTA's share of a 32-key tile
+constexpr int kStageBytes = kTileBytes;    // a ring slot: a tile share or a 16 KB query slab
 constexpr int kGroups = 3;                 // softmax groups (4 warps each) taking turns by tile
 constexpr int kXWarp = 32 * kNK * 4;       // 4 KB: one warp's 32 rows of a partial score tile
 
 constexpr int kOffKV = 0;
 constexpr int kOffX = kOffKV + kStages * kStageBytes;     // receive slots (peer → this CTA), per warp
 constexpr int kOffY = kOffX + kGroups * 4 * kXWarp;       // staging slots, one per lane quarter
-constexpr int kOffQPe = kOffY + 4 * kXWarp;               // rank 1: rotary query slab (A from smem)
-constexpr int kOffRed = kOffQPe + kSlabQ;                 // row-max / row-sum exchange
+constexpr int kOffQPe = kOffY + 4 * kXWarp;               // this CTA's rotary query columns
+constexpr int kOffRed = kOffQPe + kSlabQPe;               // row-max / row-sum exchange
 constexpr int kOffBar = kOffRed + (2 + 2 * kGroups) * 128 * 4;
 constexpr int kAttnSmem = kOffBar + 768 + 1024;
 
@@ -150,6 +155,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     latent_attention_kernel(const __grid_constant__ CUtensorMap tmKV,
                             const __grid_constant__ CUtensorMap tmPE,
                             const __grid_constant__ CUtensorMap tmQ,
+                            const __grid_constant__ CUtensorMap tmQPe,
                             const __grid_constant__ CUtensorMap tmO,
                             const __grid_constant__ CUtensorMap tmPart,
                             const __grid_constant__ CUtensorMap tmKV2,
@@ -182,9 +188,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const long long e0 = pair_begin(total, pairs, pair), e1 = pair_begin(total, pairs, pair + 1);
 
   const int warp = static_cast<int>(warp_id());
-  const int nslabs = rank == 0 ? 4 : 5;           // 64-column cache slabs this CTA owns
-  const int col0 = rank == 0 ? 0 : 256;           // first cache / query column it owns
-  uint8_t* sQPe = smem + kOffQPe;                 // rank 1: the rotary query slab
+  const int col0 = rank == 0 ? 0 : 256;           // first latent cache / query column it owns
+  const int pe0 = rank == 0 ? 0 : 32;             // first rotary column it owns
+  uint8_t* sQPe = smem + kOffQPe;                 // this CTA's rotary query columns
   Guard guard{reinterpret_cast<volatile int*>(&bar->abort_flag), p.status,
               p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs};
 
@@ -213,6 +219,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmKV);
     tma_prefetch_desc(&tmPE);
     tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmQPe);
     tma_prefetch_desc(&tmO);
     tma_prefetch_desc(&tmPart);
     if (p.topk_idx) {
@@ -293,7 +300,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           rr[i] = static_cast<int>(rowbase + t);
         }
         int s = 0;
-        if (lane == 0) s = take_slot(nslabs * kSlabKV);
+        if (lane == 0) s = take_slot(kTileBytes);
         s = __shfl_sync(0xffu, s, 0);
         if (s < 0) { ok = false; break; }
         uint64_t* fb = &bar->kv_full[s];
@@ -301,9 +308,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i)
           tma_gather4(dst + i * kSlabKV + lane * 512, &tmKV2, fb, col0 + 64 * i, rr[0], rr[1],
                       rr[2], rr[3], pol);
-        if (rank == 1)
-          tma_gather4(dst + 4 * kSlabKV + lane * 512, &tmPE2, fb, 0, rr[0], rr[1], rr[2], rr[3],
-                      pol);
+        tma_gather4(dst + 4 * kSlabKV + lane * 256, &tmPE2, fb, pe0, rr[0], rr[1], rr[2], rr[3],
+                    pol);
       }
       it.next();
     }
@@ -335,7 +341,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (pf_live && pf_key < pf_end) {
             if (kL2Every > 0 && (pf_n++ % (kL2Every > 0 ? kL2Every : 1)) == 0) {
               for (int i = 0; i < 4; ++i) tma_prefetch_l2_3d(&tmKV, col0 + 64 * i, pf_key, pf_b);
-              if (rank == 1) tma_prefetch_l2_3d(&tmPE, 0, pf_key, pf_b);
+              tma_prefetch_l2_3d(&tmPE, pe0, pf_key, pf_b);
             }
             pf_key += kNK;
             return;
@@ -376,26 +382,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tma_load_3d(sKV + s * kStageBytes, &tmQ, &bar->kv_full[s], col0 + 64 * i, 0, row);
         }
         for (int j = 0; j < ntiles && ok; ++j) {
-          const int s = take_slot(nslabs * kSlabKV);
+          const int s = take_slot(kTileBytes);
           if (s < 0) { ok = false; break; }
           uint64_t* fb = &bar->kv_full[s];
           uint8_t* dst = sKV + s * kStageBytes;
           const int key = k0 + j * kNK;
           for (int i = 0; i < 4; ++i)
             tma_load_3d_hint(dst + i * kSlabKV, &tmKV, fb, col0 + 64 * i, key, b, pol);
-          if (rank == 1) tma_load_3d_hint(dst + 4 * kSlabKV, &tmPE, fb, 0, key, b, pol);
+          tma_load_3d_hint(dst + 4 * kSlabKV, &tmPE, fb, pe0, key, b, pol);
           prefetch_next();
         }
         it.next();
       }
-    } else if (lane == qpe_lane && rank == 1) {
+    } else if (lane == qpe_lane) {
       pdl_wait();
       int row, k0, k1, nrow, pc = 0;
       bool first_row;
       while (it.get(row, k0, k1, nrow, first_row)) {
         if (pc > 0 && !mbar_wait(&bar->q_empty, (pc - 1) & 1, guard)) break;
-        mbar_arrive_expect_tx(&bar->qpe_full, kSlabQ);
-        tma_load_3d(sQPe, &tmQ, &bar->qpe_full, kC, 0, row);
+        mbar_arrive_expect_tx(&bar->qpe_full, kSlabQPe);
+        tma_load_3d(sQPe, &tmQPe, &bar->qpe_full, kC + pe0, 0, row);
         qpe_armed = ++pc;
         it.next();
       }
@@ -425,7 +431,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           umma_commit(&bar->kv_empty[s]);
         }
         if (!ok) break;
-        if (rank == 1 && !mbar_wait(&bar->qpe_full, pc & 1, guard)) break;
+        if (!mbar_wait(&bar->qpe_full, pc & 1, guard)) break;
         const int rs0 = rs;
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
           const int s = (rs0 + j) % kStages, sb = g % kNS;
@@ -436,8 +442,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          // scores: S[128 x 32] = Q_half x K_half^T: latent part with the query in TMEM, the
-          // rotary part (rank 1) with the query slab in shared memory; cache K-major in smem
+          // scores: S[128 x 32] = Q_part x K_part^T over this CTA's 256 latent and 32 rotary
+          // columns: latent part with the query in TMEM, rotary part with the query in shared
+          // memory (64-byte-swizzled 32-column slabs); cache K-major in smem
           const uint32_t kv0 = smem_u32(sKV + s * kStageBytes);
           for (int i = 0; i < 4; ++i) {
 #pragma unroll
@@ -447,12 +454,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                (i | kk) != 0);
             }
           }
-          if (rank == 1) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              umma_bf16(tmem + kTmemS + sb * kNK, smem_desc_sw128(qpe0 + kk * 32, 16, 1024),
-                        smem_desc_sw128(kv0 + 4 * kSlabKV + kk * 32, 16, 1024), idesc_qk, 1u);
-            }
+          for (int kk = 0; kk < 2; ++kk) {
+            umma_bf16(tmem + kTmemS + sb * kNK, smem_desc_sw64(qpe0 + kk * 32, 512),
+                      smem_desc_sw64(kv0 + 4 * kSlabKV + kk * 32, 512), idesc_qk, 1u);
           }
           umma_commit(&bar->s_full[g % kNB]);
           if (j == ntiles - 1) umma_commit(&bar->q_empty);
@@ -874,7 +879,7 @@ cudaError_t attention_prepare() {
 cudaError_t launch_attention(const AttnMaps& m, const AttnParams& p, int n_pairs, cudaStream_t s,
                              bool pdl) {
   LaunchCfg lc(dim3(2 * n_pairs), dim3(kThreads), kAttnSmem, s, pdl);
-  return cudaLaunchKernelEx(&lc.cfg, latent_attention_kernel, m.kv, m.pe, m.q, m.o, m.part,
+  return cudaLaunchKernelEx(&lc.cfg, latent_attention_kernel, m.kv, m.pe, m.q, m.qpe, m.o, m.part,
                             p.topk_idx ? m.kv2 : m.kv, p.topk_idx ? m.pe2 : m.pe, p);
 }
 
@@ -885,11 +890,11 @@ bool make_gather_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st,
   if (rows >= (1ull << 31)) return false;   // gather row coordinates are 32-bit
   const uint64_t d_kv[2] = {kC, rows}, s_kv[1] = {static_cast<uint64_t>(kv_st) * 2};
   const uint64_t d_pe[2] = {kDr, rows}, s_pe[1] = {static_cast<uint64_t>(pe_st) * 2};
-  const uint32_t box[2] = {64, 1};
+  const uint32_t box[2] = {64, 1}, box_pe[2] = {32, 1};
   return encode_tiled(&m->kv2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv, d_kv, s_kv, box,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
-         encode_tiled(&m->pe2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pe, d_pe, s_pe, box,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
+         encode_tiled(&m->pe2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pe, d_pe, s_pe, box_pe,
+                      CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_st, const void* pe,
@@ -900,19 +905,21 @@ bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_
   const uint64_t L = static_cast<uint64_t>(max_seq_len), Bt = static_cast<uint64_t>(batch);
   const uint64_t R = static_cast<uint64_t>(rows), H = static_cast<uint64_t>(n_heads);
   const uint32_t box_kv[3] = {64, static_cast<uint32_t>(kNK), 1};
+  const uint32_t box_pe[3] = {32, static_cast<uint32_t>(kNK), 1};   // 64-byte rows
   const uint64_t d_kv[3] = {kC, L, Bt}, s_kv[2] = {static_cast<uint64_t>(kv_st) * 2,
                                                    static_cast<uint64_t>(kv_sb) * 2};
   const uint64_t d_pe[3] = {kDr, L, Bt}, s_pe[2] = {static_cast<uint64_t>(pe_st) * 2,
                                                     static_cast<uint64_t>(pe_sb) * 2};
   const uint64_t d_q[3] = {kDk, kHPad, R}, s_q[2] = {kDk * 2, kHPad * kDk * 2};
-  const uint32_t box_q[3] = {64, 128, 1};
+  const uint32_t box_q[3] = {64, 128, 1}, box_qpe[3] = {32, 128, 1};
   const uint64_t d_o[3] = {kC, H, R}, s_o[2] = {kC * 2, H * kC * 2};
   const uint32_t box_o[3] = {64, 32, 1};
   const uint64_t d_p[2] = {kC, static_cast<uint64_t>(pairs) * 2 * 128}, s_p[1] = {kC * 2};
   const uint32_t box_p[2] = {64, 32};
   return encode_tiled(&m->kv, bf, 3, kv, d_kv, s_kv, box_kv, sw) &&
-         encode_tiled(&m->pe, bf, 3, pe, d_pe, s_pe, box_kv, sw) &&
+         encode_tiled(&m->pe, bf, 3, pe, d_pe, s_pe, box_pe, CU_TENSOR_MAP_SWIZZLE_64B) &&
          encode_tiled(&m->q, bf, 3, qabs, d_q, s_q, box_q, sw) &&
+         encode_tiled(&m->qpe, bf, 3, qabs, d_q, s_q, box_qpe, CU_TENSOR_MAP_SWIZZLE_64B) &&
          encode_tiled(&m->o, bf, 3, o_lat, d_o, s_o, box_o, sw) &&
          encode_tiled(&m->part, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, part_o, d_p, s_p, box_p, sw);
 }
