@@ -42,8 +42,8 @@
 //   * Online softmax in exp2 domain with lazy rescaling: the running max is only raised (and O
 //     in TMEM rescaled) when a tile's max exceeds it by more than 8 (factor 256), which keeps the
 //     rescale off the common path while the result stays exact.
-//   * Warp roles: warp 0 TMA producer (lane 1 of rank 1: rotary query slab; in the index-mask mode
-//     lanes 0-7 gather the cache rows by index and lane 31 loads the rotary slab), warp 1 TMEM owner
+//   * Warp roles: warp 0 TMA producer (lane 1: the CTA's rotary query columns; in the index-mask
+//     mode lanes 0-7 gather the cache rows by index and lane 31 loads the rotary query), warp 1 TMEM owner
 //     + score-MMA issuer (and the query copies), warp 2 P·V issuer, warps 3-14 softmax and
 //     epilogue (thread = head row = TMEM lane).  A tcgen05 instruction costs a single issuing
 //     thread ~48 cycles, so the score and P·V streams are issued by two threads in parallel.
@@ -101,7 +101,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_empty;         // the piece's last score MMA has read the query (TMEM and smem)
-  uint64_t qpe_full;        // rank 1: the piece's rotary query slab has landed
+  uint64_t qpe_full;        // the piece's rotary query columns (this CTA's 32) have landed
   uint64_t s_full[kNB], p_full[kNS], pv_done[kNB];
   uint64_t o_empty;
   uint64_t x_full[4 * kGroups], x_empty[4 * kGroups];   // [group][warp quad]
@@ -242,7 +242,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   for (int s = 0; s < kStages; ++s) last_slot[s] = -1;
   int qpe_armed = 0;
 
-  // lane of warp 0 that loads rank 1's rotary query slabs (lanes 0-7 gather in the index-mask
+  // lane of warp 0 that loads the CTA's rotary query columns (lanes 0-7 gather in the index-mask
   // mode)
   const uint32_t qpe_lane = p.topk_idx ? 31u : 1u;
   if (warp == 0 && p.topk_idx && lane_id() < 8) {
@@ -317,8 +317,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     // Lane 0: ring slot sequence per piece = the 4 latent query slabs this CTA owns (128 x 64
-    // columns, 16 KB each), then the piece's cache tiles.  Lane qpe_lane of rank 1: the piece's
-    // rotary query slab into its own buffer, once the previous piece's last score MMA has read it.
+    // columns, 16 KB each), then the piece's cache tiles.  Lane qpe_lane: the piece's 32 rotary
+    // query columns of this CTA into their own buffer, once the previous piece's last score MMA
+    // has read them.
     const uint32_t lane = lane_id();
     if (lane == 0 && !p.topk_idx) {
       // decode reads each cache row once (evict first); a prefill chunk's rows all re-read the
