@@ -930,69 +930,86 @@ bool make_attention_maps(AttnMaps* m, const void* kv, int64_t kv_sb, int64_t kv_
 // One warp per (row, head) task; lane l owns columns l, l+32, ..., l+480.
 // ------------------------------------------------------------------------------------------
 
-// Persistent grid (one block per SM, launched once): each warp walks (row, head) tasks.
+// Persistent grid (one block per SM, launched once): each warp walks (row, head) tasks.  Most
+// rows are uncut, so a warp first reads the piece records of its next 32 tasks at once (one per
+// lane, one round trip), then merges only the tasks whose row was cut.
 constexpr int kCombineThreads = 512;
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineParams p) {
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
-  const int warps = gridDim.x * (kCombineThreads / 32);
-  for (int task = blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5);
-       task < p.rows * p.n_heads; task += warps) {
-  const int r = task / p.n_heads, h = task - r * p.n_heads;
-  const int2 pcs = __ldcg(p.row_pieces + r);
-  const int plo = pcs.x >> 1, phi = pcs.y;
-  const int slot_lo = pcs.x & 1;   // the first piece is the tail of a pair begun in an earlier row
-  if (plo == phi) continue;   // written by one pair
-  if (plo < 0 || phi < plo || phi >= p.n_pairs) {   // not a record the key prefix can produce
-    if (lane == 0) atomicCAS(p.status, kDevOk, kDevBadArg);
-    continue;
-  }
-  // online log-sum-exp merge, four pieces' loads in flight at a time
-  constexpr int kBatch = 4;
-  float mx = -INFINITY, wsum = 0.f;
-  float acc[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  for (int q0 = plo; q0 <= phi; q0 += kBatch) {
-    float lse[kBatch], v[kBatch][16];
-#pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      const int q = q0 + b;
-      lse[b] = -INFINITY;
-      if (q <= phi) {
-        const int slot = q == plo ? slot_lo : 0;
-        const size_t base = (static_cast<size_t>(q) * 2 + slot) * 128 + h;
-        lse[b] = __ldg(p.part_lse + base);
-        const __half* src = p.part_o + base * kC;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[b][i] = __half2float(src[lane + 32 * i]);
+  const long long warps = static_cast<long long>(gridDim.x) * (kCombineThreads / 32);
+  const long long ntasks = static_cast<long long>(p.rows) * p.n_heads;
+  for (long long base = static_cast<long long>(blockIdx.x) * (kCombineThreads / 32) + (threadIdx.x >> 5);
+       base < ntasks; base += 32 * warps) {
+    // this lane's task of the batch: base + lane * warps
+    const long long mine = base + lane * warps;
+    int2 rec = make_int2(0, 0);
+    bool cut = false;
+    if (mine < ntasks) {
+      rec = __ldcg(p.row_pieces + mine / p.n_heads);
+      const int plo = rec.x >> 1, phi = rec.y;
+      if (plo < 0 || phi < plo || phi >= p.n_pairs) {   // not a record the key prefix can produce
+        atomicCAS(p.status, kDevOk, kDevBadArg);
+      } else {
+        cut = plo != phi;   // an uncut row was written by one pair
       }
     }
-    float m_new = mx;
+    unsigned todo = __ballot_sync(0xffffffffu, cut);
+    while (todo) {
+      const int src = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const long long task = base + src * warps;
+      const int r = static_cast<int>(task / p.n_heads), h = static_cast<int>(task - static_cast<long long>(r) * p.n_heads);
+      const int rx = __shfl_sync(0xffffffffu, rec.x, src), ry = __shfl_sync(0xffffffffu, rec.y, src);
+      const int plo = rx >> 1, phi = ry;
+      const int slot_lo = rx & 1;   // the first piece is the tail of a pair begun in an earlier row
+      // online log-sum-exp merge, four pieces' loads in flight at a time
+      constexpr int kBatch = 4;
+      float mx = -INFINITY, wsum = 0.f;
+      float acc[16];
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) m_new = fmaxf(m_new, lse[b]);
-    const float f = mx == -INFINITY ? 0.f : exp2f((mx - m_new) * 1.4426950408889634f);
-    wsum *= f;
+      for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+      for (int q0 = plo; q0 <= phi; q0 += kBatch) {
+        float lse[kBatch], v[kBatch][16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) acc[i] *= f;
+        for (int b = 0; b < kBatch; ++b) {
+          const int q = q0 + b;
+          lse[b] = -INFINITY;
+          if (q <= phi) {
+            const int slot = q == plo ? slot_lo : 0;
+            const size_t pbase = (static_cast<size_t>(q) * 2 + slot) * 128 + h;
+            lse[b] = __ldg(p.part_lse + pbase);
+            const __half* psrc = p.part_o + pbase * kC;
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      if (q0 + b <= phi) {
-        const float w = exp2f((lse[b] - m_new) * 1.4426950408889634f);
-        wsum += w;
+            for (int i = 0; i < 16; ++i) v[b][i] = __half2float(psrc[lane + 32 * i]);
+          }
+        }
+        float m_new = mx;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = fmaf(w, v[b][i], acc[i]);
+        for (int b = 0; b < kBatch; ++b) m_new = fmaxf(m_new, lse[b]);
+        const float f = mx == -INFINITY ? 0.f : exp2f((mx - m_new) * 1.4426950408889634f);
+        wsum *= f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] *= f;
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+          if (q0 + b <= phi) {
+            const float w = exp2f((lse[b] - m_new) * 1.4426950408889634f);
+            wsum += w;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[i] = fmaf(w, v[b][i], acc[i]);
+          }
+        }
+        mx = m_new;
       }
-    }
-    mx = m_new;
-  }
-  const float inv = 1.f / wsum;
-  bf16* dst = p.o_lat + (static_cast<size_t>(r) * p.n_heads + h) * kC;
+      const float inv = 1.f / wsum;
+      bf16* dst = p.o_lat + (static_cast<size_t>(r) * p.n_heads + h) * kC;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) dst[lane + 32 * i] = __float2bfloat16_rn(acc[i] * inv);
-  if (lane == 0 && p.lse_out) p.lse_out[static_cast<size_t>(r) * p.n_heads + h] = mx + logf(wsum);
+      for (int i = 0; i < 16; ++i) dst[lane + 32 * i] = __float2bfloat16_rn(acc[i] * inv);
+      if (lane == 0 && p.lse_out) p.lse_out[static_cast<size_t>(r) * p.n_heads + h] = mx + logf(wsum);
+    }
   }
 }
 
