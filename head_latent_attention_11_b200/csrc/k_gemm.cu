@@ -17,8 +17,9 @@
 //   warp 1      allocates TMEM and issues tcgen05.mma (M=128, N=BN, K=16) per slab into one of
 //               two accumulators (units alternate), committing each slab back to the producer
 //               and each finished unit to the epilogue;
-//   warps 2-9   epilogue, two warps per TMEM lane quadrant (warp % 4) splitting the 16-token
-//               blocks: tcgen05.ld the fp32 accumulator (thread = weight row), apply RoPE for
+//   warps 2-..  epilogue, four warps per TMEM lane quadrant (warp % 4) splitting the 16-token
+//               blocks (two in the merge and FP8 modes, which need the registers): tcgen05.ld
+//               the fp32 accumulator (thread = weight row), apply RoPE for
 //               the rotary rows of wq_b (partner of a pair = neighbouring lane), transpose 16
 //               tokens at a time through shared memory and store bf16 as 16-byte vectors (8
 //               consecutive rows of one token), hand the accumulator back — overlapping the next
@@ -32,8 +33,14 @@ namespace mla {
 
 namespace {
 
-constexpr int kEpiWarps = 8;                            // two per TMEM lane quadrant
+// Epilogue warps: the epilogue of a 128 x 256 tile is a chain of 16-token blocks per warp
+// (tcgen05.ld, transpose through shared memory, 16-byte stores) and paces large-N GEMMs, so the
+// plain bf16 kernel runs four warps per TMEM lane quadrant.  The merge and FP8 modes keep two
+// (their B builder and converters need the registers of a smaller block).
+constexpr int kEpiWarps = 8;                            // merge / FP8 modes
 constexpr int kEpiThreads = 32 * kEpiWarps;
+template <bool FP8, bool MERGE>
+__host__ __device__ constexpr int epi_warps() { return (FP8 || MERGE) ? kEpiWarps : 2 * kEpiWarps; }
 // FP8: converter threads — four warps; two in the merge mode, whose B builder needs the registers
 // (a block of more than 384 threads is held to 128 registers a thread)
 template <bool MERGE>
@@ -42,7 +49,7 @@ constexpr int kSlabA = 128 * 64 * 2;   // 16 KB
 constexpr int kSlabA8 = 128 * 64;      // 8 KB: an FP8 weight slab (64-byte rows, no swizzle)
 
 template <bool FP8, bool MERGE = false>
-constexpr int gemm_threads() { return 64 + kEpiThreads + (FP8 ? conv_threads<MERGE>() : 0); }
+constexpr int gemm_threads() { return 64 + 32 * epi_warps<FP8, MERGE>() + (FP8 ? conv_threads<MERGE>() : 0); }
 
 template <int BN>
 struct GemmTile {
@@ -56,13 +63,13 @@ constexpr int kMergeSlabs = kC / 64;
 
 // Plain-store epilogue: each epilogue warp transposes its 32 rows x 16 tokens of bf16 through a
 // 1 KB staging block so that the global writes are 16-byte vectors.
-constexpr int kEpiStageBytes = kEpiWarps * 32 * 16 * 2;
+constexpr int kEpiWarpStage = 32 * 16 * 2;
 
 template <int BN, int STAGES, bool MERGE = false, bool FP8 = false>
 constexpr int gemm_smem_bytes() {
   return 1024 /*align slack*/ + STAGES * kSlabA +
          (MERGE ? kMergeSlabs * GemmTile<BN>::kSlabB : STAGES * GemmTile<BN>::kSlabB) +
-         (FP8 ? STAGES * kSlabA8 : 0) + 512 /*barriers*/ + kEpiStageBytes;
+         (FP8 ? STAGES * kSlabA8 : 0) + 512 /*barriers*/ + epi_warps<FP8, MERGE>() * kEpiWarpStage;
 }
 
 // 16 FP8 E4M3 codes (bytes of v, lowest first) times `scale` → 16 bf16 (lo: codes 0-7).
@@ -356,7 +363,7 @@ __global__ void __launch_bounds__(gemm_threads<FP8, MERGE>(), 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], kEpiThreads);
+      mbar_init(&acc_empty[i], 32 * epi_warps<FP8, MERGE>());
     }
     mbar_init(drain, 1);
     mbar_init(b_ready, kEpiThreads);
@@ -447,14 +454,14 @@ __global__ void __launch_bounds__(gemm_threads<FP8, MERGE>(), 1)
       }
       umma_commit(drain);
     }
-  } else if (FP8 && warp >= 2 + kEpiWarps) {
+  } else if (FP8 && warp >= 2 + epi_warps<FP8, MERGE>()) {
     // FP8 converter warps: each ring slab of fp8 weight codes → bf16 (code × the block's scale)
     // in the 128-byte-swizzled layout the MMA reads; thread t converts 16-byte chunks t, t + T,
     // t + 2T, ... of the slab (T converter threads; row = chunk / 4, 16 columns each).  A slab (128 rows x 64
     // columns) lies in one 128 x 128 scale block.  Lane b of every converter warp holds the scale
     // of K block b of the current tile and has the next tile's in flight, so no slab waits on a
     // scale load (the launcher limits FP8 GEMMs to K <= 32 * 128).
-    const int ctid = static_cast<int>(threadIdx.x) - (64 + kEpiThreads);
+    const int ctid = static_cast<int>(threadIdx.x) - (64 + 32 * epi_warps<FP8, MERGE>());
     const int lane = static_cast<int>(lane_id());
     const int kblocks = (p.K + 127) / 128;
     auto tile_scale = [&](int unit) -> float {   // this lane's K block of tile `unit`
@@ -498,13 +505,14 @@ __global__ void __launch_bounds__(gemm_threads<FP8, MERGE>(), 1)
       }
     }
   } else {
-    // epilogue warps 2 .. 1+kEpiWarps → TMEM lane quadrant warp % 4
+    // epilogue warps 2 .. 1 + epi_warps → TMEM lane quadrant warp % 4
     pdl_wait();   // outputs may be read by the kernel before this one
     const int quad = warp & 3;
     const int row = quad * 32 + static_cast<int>(lane_id());
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const int etid = static_cast<int>(threadIdx.x) - 64;   // 0 .. kEpiThreads-1
-    const int half = etid >> 7;   // the two warps of a lane quadrant split the 16-token blocks
+    const int etid = static_cast<int>(threadIdx.x) - 64;   // 0 .. 32 * epi_warps - 1
+    constexpr int kSub = epi_warps<FP8, MERGE>() / 4;       // warps per lane quadrant
+    const int sub = etid >> 7;    // the warps of a lane quadrant split the 16-token blocks
     // the epilogue writes 16-byte vectors: every 8-row group must start 16-byte aligned (the C
     // ABI requires aligned outputs; a violation is reported, never written)
     const bool aligned_out =
@@ -532,7 +540,7 @@ __global__ void __launch_bounds__(gemm_threads<FP8, MERGE>(), 1)
       __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sEpi + (warp - 2) * 1024);
       const int mw = un.m0 + quad * 32;   // first row of this warp
 #pragma unroll 1
-      for (int c0 = 16 * half; c0 < BN; c0 += 32) {
+      for (int c0 = 16 * sub; c0 < BN; c0 += 16 * kSub) {
         if (un.n0 + c0 >= p.N) break;   // uniform across the warp
         float v[16];
         float2 cs[16];
