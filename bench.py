@@ -94,19 +94,30 @@ def measured_peaks() -> dict:
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+# The attention kernel's part of k_attn.cu: everything before the combine kernel's section (the
+# combine is a separate launch and does not change the attention's traffic).
+ATTN_SOURCE_END = b"// Combine: rows cut between pairs merge"
+
+
+def attention_source_sha256() -> str:
+    """sha256 of the attention kernel's source region of k_attn.cu."""
+    import hashlib
+    src = os.path.join(ROOT, "head_latent_attention_11_b200", "csrc", "k_attn.cu")
+    with open(src, "rb") as f:
+        text = f.read()
+    cut = text.find(ATTN_SOURCE_END)
+    return hashlib.sha256(text[:cut] if cut >= 0 else text).hexdigest()
+
+
 def profiled_traffic(workload_name: str):
     """DRAM bytes (read + write) of one attention launch from the committed ncu summary, or None
     when there is none for this workload or the kernel source changed since it was captured."""
-    import hashlib
     prof = os.path.join(ROOT, "profiles", f"latent_attention_{workload_name}.json")
-    src = os.path.join(ROOT, "head_latent_attention_11_b200", "csrc", "k_attn.cu")
-    if not (os.path.exists(prof) and os.path.exists(src)):
+    if not os.path.exists(prof):
         return None
     with open(prof) as f:
         d = json.load(f)
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    if not sha.startswith(d.get("source_sha256_prefix", "-")):
+    if not attention_source_sha256().startswith(d.get("source_sha256_prefix", "-")):
         return None
     return int(d["dram_bytes_read"]) + int(d["dram_bytes_write"])
 
