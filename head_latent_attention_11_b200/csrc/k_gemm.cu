@@ -539,6 +539,7 @@ __global__ void __launch_bounds__(gemm_threads<FP8, MERGE>(), 1)
       // [token][32 rows], then each lane writes two 16-byte pieces (8 rows of one token)
       __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sEpi + (warp - 2) * 1024);
       const int mw = un.m0 + quad * 32;   // first row of this warp
+      const bool rope_epi = p.epi == kEpiWqbRope;   // only the rotary rows need the partner row
 #pragma unroll 1
       for (int c0 = 16 * sub; c0 < BN; c0 += 16 * kSub) {
         if (un.n0 + c0 >= p.N) break;   // uniform across the warp
@@ -548,7 +549,7 @@ __global__ void __launch_bounds__(gemm_threads<FP8, MERGE>(), 1)
         tmem_ld16(tmem + lane_off + ab * BN + c0, v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float partner = __shfl_xor_sync(0xffffffffu, v[i], 1);
+          const float partner = rope_epi ? __shfl_xor_sync(0xffffffffu, v[i], 1) : 0.f;
           stg[i * 32 + lane_id()] = __float2bfloat16_rn(epi_value(p, m, v[i], partner, cs[i]));
         }
         __syncwarp();
