@@ -272,15 +272,6 @@ __host__ __device__ inline long long pair_begin(long long total_keys, int pairs,
   return total_keys * p / pairs;
 }
 
-// Pair whose key range contains flattened key e.
-__host__ __device__ inline int pair_of_key(long long total, int pairs, long long e) {
-  int q = static_cast<int>((e * pairs) / total);
-  if (q >= pairs) q = pairs - 1;
-  while (q + 1 < pairs && pair_begin(total, pairs, q + 1) <= e) ++q;
-  while (q > 0 && pair_begin(total, pairs, q) > e) --q;
-  return q;
-}
-
 // Row containing flattened key e: largest r with prefix[r] <= e (plain loads: the prefix may
 // have been written earlier by the calling kernel).
 __device__ __forceinline__ int row_of_key(const long long* prefix, int rows, long long e) {
