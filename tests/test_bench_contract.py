@@ -73,3 +73,29 @@ def test_algorithmic_work_matches_the_hand_count():
     assert wk["cache_bytes"] == (2048 + 2048) * 1152
     t = np.arange(2048)
     assert wk["keys"] == int((2048 + t + 1).sum())
+
+
+def test_recorded_traffic_follows_the_attention_source_only(tmp_path, monkeypatch):
+    """The DRAM bytes of a committed ncu record are reported only while the attention kernel's
+    source region (k_attn.cu before the combine kernel's section) is the one recorded: an edit to
+    the combine kernel keeps the record, an edit to the attention kernel voids it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    src = os.path.join(ROOT, "head_latent_attention_11_b200", "csrc", "k_attn.cu")
+    text = open(src, "rb").read()
+    cut = text.find(bench.ATTN_SOURCE_END)
+    assert cut > 0, "the combine section marker is missing from k_attn.cu"
+    (tmp_path / "head_latent_attention_11_b200" / "csrc").mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    kattn = tmp_path / "head_latent_attention_11_b200" / "csrc" / "k_attn.cu"
+    kattn.write_bytes(text)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    rec = {"source_sha256_prefix": bench.attention_source_sha256()[:16],
+           "dram_bytes_read": 1000, "dram_bytes_write": 24}
+    (tmp_path / "profiles" / "latent_attention_x.json").write_text(json.dumps(rec))
+    assert bench.profiled_traffic("x") == 1024
+    kattn.write_bytes(text + b"\n// a later change to the combine kernel\n")
+    assert bench.profiled_traffic("x") == 1024
+    kattn.write_bytes(text[:cut] + b"// a change to the attention kernel\n" + text[cut:])
+    assert bench.profiled_traffic("x") is None
+    assert bench.profiled_traffic("missing") is None
